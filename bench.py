@@ -1,0 +1,362 @@
+"""Benchmark of the CSA/HCA hot path on B200: decode queries/s and roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c1] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+for a CSA workload csa_compress (the block the step completes) ->
+csa_index_topk -> csa_sparse_attn; for an HCA workload hca_compress ->
+hca_dense_attn.  The default workload is the V4-Flash-shaped CSA decode
+(batch 32, 131072-token context, 32768 entries, top-512, 64 heads).
+
+Timing: W untimed warm-up steps, then exactly K steps between CUDA events on
+the launching stream, bracketed by a barrier and torch.cuda.synchronize().
+The timed loop rotates over several device-resident copies of the workload
+so that the bytes one cycle touches exceed 3x the L2 size: every step reads
+its inputs from HBM, no flush is needed.  Multi-GPU (torchrun): every rank
+runs the same per-GPU workload (weak scaling) with no data-path collective;
+the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only other program here that
+runs the same method) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "CSA/HCA decode queries/s at 128K-1M ctx; % of HBM / tensor-core roofline"
+L2_BYTES = 126 * 2 ** 20
+
+CONFIG_NAMES = {
+    "c0": "tiny CSA decode fp32 (B=1, L=2048, d=128)",
+    "c1": "V4-Flash-shaped CSA decode (B=32, L=131072, N=32768, top-512, n_h=64, d=512 FP8+BF16, MXFP4 indexer 64x128)",
+    "c2": "V4-Pro-shaped CSA decode (B=4, L=1048576, N=262144, top-1024, n_h=128, planted cluster)",
+    "c3": "HCA decode (B=16, L=1048576, m=128, N=8192, n_h=128, dense)",
+    "c4": "CSA chunked prefill (B=2, T=32768, N=8192, top-512, n_h=64)",
+}
+
+
+def algorithmic_bytes(w):
+    """Bytes the method must move per step, and those of the dominant call.
+
+    Per query of a CSA decode: every visible index key (c/2 + c/32 bytes),
+    the index query + weights, the k selected entries and W window rows
+    (d + r + 4 bytes each), the query and the output (n_h*d*2 each), the
+    k indices; plus the compressor's 2m stream rows and gates and its
+    written entry.  HCA: every visible entry instead of keys/selection.
+    Returns (step_bytes, index_call_bytes).
+    """
+    p = w["params"]
+    B, T = p.B, w["T"]
+    row = p.d + p.r + 4 if p.kv_fmt == "fp8" else 4 * p.d
+    act = 2 if p.act_fmt == "bf16" else 4
+    key = p.c_I // 2 + p.c_I // 32 if p.idx_fmt == "mxfp4" else 4 * p.c_I
+    step = idx_call = 0
+    for b in range(B):
+        for tq in range(T):
+            t = int(w["q_pos0"][b]) + tq
+            n_t = min((t + 1) // p.m, w["Ncap"])
+            win = min(p.W, t + 1)
+            qo = 2 * p.n_h * p.d * act
+            if p.k > 0:
+                iq = p.H_I * key + 4 * p.H_I
+                ic = n_t * key + iq + 4 * p.k
+                idx_call += ic
+                step += ic + (min(p.k, n_t) + win) * row + qo + 4 * p.k
+            else:
+                step += (n_t + win) * row + qo
+    if w["S"]:
+        ne = int((np.asarray(w["e_end"]) - np.asarray(w["e_begin"])).sum())
+        step += ne * (2 * p.m * p.d * act + 2 * p.m * 4 + row + 4)
+    return step, idx_call
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out = self.proc.communicate(timeout=10)[0]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def oracle_sample(w, n_queries):
+    """Time the oracle on the first n_queries queries of the workload."""
+    from oracle import pipeline
+    p = w["params"]
+    qs = [(b, tq) for b in range(p.B) for tq in range(w["T"])][:n_queries]
+    seqs = sorted(set(b for b, _ in qs))
+    t0 = time.perf_counter()
+    comp = pipeline.compress(w, seqs=seqs) if w["S"] else None
+    if p.k > 0:
+        idx = pipeline.index_topk(w, qs)
+        pipeline.sparse_attn(w, idx, comp, qs)
+    else:
+        pipeline.dense_attn(w, comp, qs)
+    return time.perf_counter() - t0, len(qs)
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.config(args.config)
+    n = {"c0": 1, "c1": 4, "c2": 1, "c3": 4, "c4": 16}[args.config]
+    for _ in range(args.warmup and 1):
+        oracle_sample(w, 1)
+    times = []
+    for _ in range(args.steps):
+        dt, nq = oracle_sample(w, n)
+        times.append(dt)
+    total = sum(times)
+    qps = args.steps * n / total
+    line = {"impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": CONFIG_NAMES[args.config], "name": args.config,
+                                            "sample_queries_per_step": n},
+            "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": f"first {n} queries of the workload per step (oracle: numpy fp64)"},
+            "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="c1", choices=sorted(CONFIG_NAMES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from long_context_sparse_gated_b200 import build, lib
+    from long_context_sparse_gated_b200.runner import STEP_INPUTS, DeviceWorkload
+    if rank == 0 or world == 1:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    lib()
+
+    seed_off = 1000 * rank
+    w = synth.config(args.config, seed={"c0": 0, "c1": 1, "c2": 2, "c3": 3, "c4": 4}[args.config] + seed_off)
+    step_bytes, idx_bytes = algorithmic_bytes(w)
+    n_copies = max(1, int(np.ceil(3 * L2_BYTES / step_bytes)))
+    if args.config == "c4":
+        n_copies = 1  # prefill touches far more than L2 per step
+    dws = [DeviceWorkload(w) for _ in range(n_copies)]
+    p = w["params"]
+    queries = p.B * w["T"]
+    stream = torch.cuda.current_stream()
+
+    def step(dw, ev=None):
+        dw.compress()
+        if p.k > 0:
+            if ev is not None:
+                ev[0].record(stream)
+            dw.index_topk()
+            if ev is not None:
+                ev[1].record(stream)
+            dw.sparse_attn()
+        else:
+            if ev is not None:
+                ev[0].record(stream)
+            dw.dense_attn()
+            if ev is not None:
+                ev[1].record(stream)
+
+    for i in range(args.warmup):
+        step(dws[i % n_copies])
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # keep the GPU busy while the sampler starts (untimed)
+    t_end = time.perf_counter() + 0.5
+    i = 0
+    while time.perf_counter() < t_end:
+        step(dws[i % n_copies])
+        i += 1
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(dws[i % n_copies], evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    kern_ms = [a.elapsed_time(b) for a, b in evs]
+    # a little more load for the clock sampler, then stop it (untimed)
+    t_end = time.perf_counter() + 0.3
+    while time.perf_counter() < t_end:
+        step(dws[i % n_copies])
+        i += 1
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    # ---- end to end: per-step inputs from pinned host memory, results back --
+    dw = dws[0]
+    host_in = {k: getattr(dw, k if k != "w_idx" else "w_idx").cpu().pin_memory()
+               for k in STEP_INPUTS if getattr(dw, k, None) is not None}
+    host_out = dw.out.cpu().pin_memory()
+    host_idx = dw.idx.cpu().pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size() + (host_idx.numel() * 4 if p.k > 0 else 0)
+
+    def e2e_step():
+        for k, t in host_in.items():
+            getattr(dw, k).copy_(t, non_blocking=True)
+        step(dw)
+        host_out.copy_(dw.out, non_blocking=True)
+        if p.k > 0:
+            host_idx.copy_(dw.idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(10, min(args.steps, 200))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms, float(np.mean(kern_ms))], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_ms, kmean = (float(x) for x in tt.tolist())
+    else:
+        kmean = float(np.mean(kern_ms))
+    err = int(sum(d.err_bits() for d in dws))
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    ms_per_step = ms / args.steps
+    value = world * queries / (ms_per_step * 1e-3)
+    peak, peak_kind = measured_peaks()
+    dom_bytes = idx_bytes if p.k > 0 else step_bytes
+    achieved = dom_bytes / (kmean * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8/bf16 storage, mxfp4 indexer, fp32 accumulate" if p.kv_fmt == "fp8" else "f32",
+        "data": "synthetic",
+        "config": {"workload": CONFIG_NAMES[args.config], "name": args.config, "batch": p.B,
+                   "context": int(w["L"].max()), "queries_per_step": queries,
+                   "l2": f"inputs larger than L2: {n_copies} device copies rotated, {n_copies * step_bytes / 2**20:.0f} MiB per cycle"},
+        "gpu_launches": args.steps * (5 if p.k > 0 else 3),
+        "roofline": {"bound": "hbm", "kernel": "csa_index_topk" if p.k > 0 else "hca_dense_attn",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": peak_kind, "traffic": None,
+                     "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean},
+        "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
+                          "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak},
+        "e2e": {"value": world * queries / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+        "device_err_bits": err,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        n = {"c0": 1, "c1": 4, "c2": 1, "c3": 4, "c4": 16}[args.config]
+        dt, nq = oracle_sample(w, n)
+        line["cpu_baseline"] = {"value": nq / dt, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                                "sample": f"first {nq} queries of the workload (numpy fp64 oracle, {dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,226 @@
+/*
+ * csa.h -- C ABI of the B200 (sm_100a) CSA/HCA hot-path library, libcsa.so.
+ *
+ * DeepSeek-V4's hybrid compressed attention, as the public write-ups of the
+ * DeepSeek-V4 technical report describe it:
+ *
+ *   csa_compress / hca_compress  gated two-stream token compressor (m = 4 for
+ *                                CSA, m = 128 for HCA), RMSNorm, partial
+ *                                RoPE, packed into the mixed FP8/BF16 layout
+ *   csa_index_topk               Lightning Indexer (FP4 block-scaled QK,
+ *                                ReLU-weighted head sum) + exact top-k
+ *   csa_sparse_attn              MQA over the selected entries + sliding
+ *                                window + attention sink, inverse RoPE
+ *   hca_dense_attn               the same attention over every entry
+ *
+ * Sources, by page title and section:
+ *   [kwkr]    kwkr.cn DeepSeek-V4 notes, 3.1 CSA 的工作方式, 3.2 HCA 的工作方式,
+ *             3.3 层间排布与滑窗补充, 3.4 两个降开销的设计, 4.4 FP4 QAT 与 KV Cache 层级
+ *   [Qiaomu]  乔木博客 "DeepSeek-V4论文解析：百万上下文、水平接近闭源模型是如何做到的？",
+ *             混合注意力机制, FP4量化感知训练, 训练配置
+ *   [WeChat]  未来科技 article on DeepSeek-V4 (cdjax.com), 1.1 混合注意力
+ *   [PACMAN]  "DeepSeek-V4 技术报告分享" talk notes (10100.com), 3.1 CSA, 3.2 HCA
+ *   [fengweifeng] "DeepSeek-V4: Towards Highly Efficient Million-Token Context
+ *             Intelligence" notes, 2. 技术实现与架构细节 (inverse RoPE offset -i)
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Pointers are DEVICE pointers unless stated otherwise; `params` is a HOST
+ *   pointer read only during the call.  `stream` is a cudaStream_t passed as
+ *   void* (NULL = the legacy default stream).  Every call only enqueues work
+ *   on `stream`; nothing synchronises and nothing is allocated: the caller
+ *   owns every buffer, including the workspace.  Calls hold no global
+ *   mutable state and are re-entrant.
+ * - Every array is C-contiguous.  The caller keeps buffers alive until the
+ *   enqueued work completes.
+ * - Return value: host-side validation only (csa_status).  Nothing is
+ *   launched when it is not CSA_OK.  Anomalies found on the device (an index
+ *   out of range, a token outside the stream buffer) are OR-ed as
+ *   CSA_DEV_ERR_* bits into *err (nullable) and the offending item is
+ *   skipped; the device never traps.
+ * - Every pointer must be 16-byte aligned (CSA_ERR_ALIGN).
+ *
+ * Storage formats
+ * ---------------
+ * KV row, CSA_KV_FP8_BF16 ([WeChat 1.1]: RoPE dims BF16, other dims FP8):
+ *     bytes [0, d-r)      E4M3 codes of the non-RoPE dims (value = code*scale)
+ *     bytes [d-r, d+r)    r BF16 values of the RoPE dims
+ *   row_bytes = d + r (576 for d = 512, r = 64); one fp32 scale per row in a
+ *   separate array.  CSA_KV_F32: d floats per row (row_bytes = 4d), no scale.
+ * Index key / index query, CSA_IDX_MXFP4 (OCP MX, E2M1 elements + UE8M0 scale
+ *   per 32): idx_dim/2 bytes, element 2i in the low nibble of byte i, plus
+ *   idx_dim/32 scale bytes in a separate array.  CSA_IDX_F32: idx_dim floats.
+ * Activations (streams, queries, outputs), CSA_ACT_BF16 or CSA_ACT_F32.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes (return values) ------------------------------------- */
+typedef int32_t csa_status;
+#define CSA_OK 0
+#define CSA_ERR_INVALID -1     /* null pointer, bad size or count            */
+#define CSA_ERR_UNSUPPORTED -2 /* shape/format outside the supported set     */
+#define CSA_ERR_ALIGN -3       /* a pointer is not 16-byte aligned           */
+#define CSA_ERR_WORKSPACE -4   /* ws too small (see the *_workspace_bytes)   */
+#define CSA_ERR_LAUNCH -5      /* a kernel launch failed (cudaGetLastError)  */
+
+/* ---- device anomaly bits, OR-ed into *err ------------------------------ */
+#define CSA_DEV_ERR_INDEX 1  /* a top-k index >= visible entries or < -1   */
+#define CSA_DEV_ERR_RANGE 2  /* a token/entry range outside its buffer     */
+
+/* ---- formats ------------------------------------------------------------ */
+#define CSA_KV_F32 0
+#define CSA_KV_FP8_BF16 1
+#define CSA_IDX_F32 0
+#define CSA_IDX_MXFP4 1
+#define CSA_ACT_F32 0
+#define CSA_ACT_BF16 1
+
+/* Layer configuration (host struct, plain old data).
+ *   B            sequences in the batch
+ *   d, r         entry dim and RoPE dims (the last r dims; r even, r <= d);
+ *                supported: d in {128, 512}, r multiple of 4, 0 < r < d
+ *   m            compression ratio: 4 (CSA) or 128 (HCA); 1..256 accepted
+ *   n_idx_heads  indexer heads H_I (1..64); idx_dim its dim c_I (64 or 128)
+ *   topk         k (1..2048) -- entries kept per query
+ *   n_heads      query heads n_h (1..128)
+ *   window       sliding-window length W in raw tokens (1..1024)
+ *   kv_fmt, idx_fmt, act_fmt   CSA_KV_*, CSA_IDX_*, CSA_ACT_*
+ *   softmax_scale  tau (logit = tau * q.v)
+ *   rope_theta     RoPE base (pair j of the last r dims turns by
+ *                  pos * theta^(-2j/r))
+ *   eps            RMSNorm epsilon
+ */
+typedef struct csa_params {
+  int32_t B, d, r, m;
+  int32_t n_idx_heads, idx_dim;
+  int32_t topk, n_heads, window;
+  int32_t kv_fmt, idx_fmt, act_fmt;
+  float softmax_scale, rope_theta, eps;
+} csa_params;
+
+/* A KV-row buffer: the compressed-entry cache, or the raw-token window ring.
+ *   rows   [B][cap][row_bytes]   (row layout above)
+ *   scale  [B][cap] fp32         (CSA_KV_FP8_BF16 only; NULL for CSA_KV_F32)
+ *   cap    rows per sequence.  For the cache, entry i of sequence b is row i.
+ *          For the window ring, the token at position p is row p mod cap. */
+typedef struct csa_kv {
+  void* rows;
+  float* scale;
+  int64_t cap;
+} csa_kv;
+
+/* ------------------------------------------------------------------------
+ * csa_compress / hca_compress  [kwkr 3.1, 3.2; Qiaomu 混合注意力机制;
+ *                               WeChat 1.1; PACMAN 3.1, 3.2]
+ *
+ * For every sequence b and entry e in [e_begin[b], e_end[b]):
+ *   logits  ga_u (u in block e: tokens m*e .. m*e+m-1, stream a) and
+ *           gb_u (u in block e-1, stream b; empty for e = 0)
+ *   w       = softmax over the union of those <= 2m logits
+ *   x       = sum_u w_u a_u + sum_u w_u b_u
+ *   y       = norm_w * x / sqrt(mean(x^2) + eps)
+ *   entry   = y with pair j of the last r dims rotated by (m*e)*theta^(-2j/r)
+ * and stores it as row e of `out` (FP8: scale = amax_nope/448, codes =
+ * E4M3 RNE-satfinite of x/scale; RoPE dims BF16 RNE), out_pos[b*cap+e] = m*e.
+ *
+ *   a, b       [B][S][d] streams (act_fmt), token at absolute position p of
+ *              sequence b is row p - tok_base[b]
+ *   gate       [B][S][2] fp32 logits (column 0: stream a, column 1: stream b)
+ *   tok_base, e_begin, e_end   int32 [B] (device)
+ *   max_entries  host upper bound on e_end[b]-e_begin[b] (sizes the grid)
+ *   norm_w     [d] fp32 RMSNorm weight, or NULL for ones
+ *   out_pos    int32 [B][out.cap], nullable
+ * Entries whose tokens fall outside [tok_base, tok_base+S) or whose slot is
+ * >= out.cap are skipped with CSA_DEV_ERR_RANGE.  csa_compress and
+ * hca_compress are the same operator; each is tuned for its own m.
+ * ---------------------------------------------------------------------- */
+csa_status csa_compress(const csa_params* params, const void* a, const void* b,
+                        const float* gate, int64_t S, const int32_t* tok_base,
+                        const int32_t* e_begin, const int32_t* e_end,
+                        int32_t max_entries, const float* norm_w, csa_kv out,
+                        int32_t* out_pos, int32_t* err, void* stream);
+csa_status hca_compress(const csa_params* params, const void* a, const void* b,
+                        const float* gate, int64_t S, const int32_t* tok_base,
+                        const int32_t* e_begin, const int32_t* e_end,
+                        int32_t max_entries, const float* norm_w, csa_kv out,
+                        int32_t* out_pos, int32_t* err, void* stream);
+
+/* ------------------------------------------------------------------------
+ * csa_index_topk  [Qiaomu 混合注意力机制, FP4量化感知训练; kwkr 3.4, 4.4;
+ *                  PACMAN 3.1]
+ *
+ * Query tau of sequence b sits at position t = q_pos0[b] + tau (tau < T)
+ * and sees the n_t = floor((t+1)/m) entries whose last token is <= t.
+ *   I(t, s) = sum_h w[b,tau,h] * max(0, q_idx[b,tau,h,:] . k_idx[b,s,:])
+ * for s < n_t, then out_idx[b][tau][0..k) = the min(k, n_t) entries with
+ * the largest I (ties -> lower s), in ascending order, padded with -1.
+ *
+ *   q_idx     [B][T][H_I] index queries (MXFP4 bytes or f32), q_idx_sf
+ *             [B][T][H_I][c_I/32] UE8M0 scales (MXFP4 only, else NULL)
+ *   w         [B][T][H_I] fp32 head weights
+ *   k_idx     [B][k_cap] index keys, k_idx_sf [B][k_cap][c_I/32]
+ *   n_max     host upper bound on n_t over the batch (<= k_cap)
+ *   out_idx   int32 [B][T][k]
+ *   ws        workspace of csa_index_topk_workspace_bytes(params, T, n_max)
+ * ---------------------------------------------------------------------- */
+csa_status csa_index_topk(const csa_params* params, const void* q_idx,
+                          const uint8_t* q_idx_sf, const float* w,
+                          const void* k_idx, const uint8_t* k_idx_sf,
+                          int64_t k_cap, const int32_t* q_pos0, int32_t T,
+                          int32_t n_max, int32_t* out_idx, void* ws,
+                          size_t ws_bytes, int32_t* err, void* stream);
+size_t csa_index_topk_workspace_bytes(const csa_params* params, int32_t T,
+                                      int32_t n_max);
+
+/* ------------------------------------------------------------------------
+ * csa_sparse_attn  [WeChat 1.1; kwkr 3.3; fengweifeng 2.; Qiaomu 混合注意力机制]
+ *
+ * For query tau of sequence b at t = q_pos0[b] + tau, head h:
+ *   J      = {cache row idx[b,tau,j] : idx >= 0} followed by the window
+ *            tokens max(0, t-W+1) .. t (ring row p mod win.cap)
+ *   z_j    = softmax_scale * q[b,tau,h,:] . v_j     (v_j is key and value)
+ *   p_j    = exp(z_j) / (exp(sink[h]) + sum_j exp(z_j))
+ *   o      = sum_j p_j v_j, the last r dims then rotated by angle -t
+ *            pair-wise (pair j by -t*theta^(-2j/r)); written in act_fmt.
+ *   q, out [B][T][n_h][d]; idx int32 [B][T][k]; sink fp32 [n_h]
+ * An idx value >= the cache capacity or < -1 is skipped with
+ * CSA_DEV_ERR_INDEX.  The window ring must hold every position in
+ * [max(0, q_pos0-W+1), q_pos0+T-1] (win.cap >= W + T - 1 suffices).
+ * ---------------------------------------------------------------------- */
+csa_status csa_sparse_attn(const csa_params* params, const void* q,
+                           csa_kv cache, const int32_t* idx, csa_kv win,
+                           const float* sink, const int32_t* q_pos0, int32_t T,
+                           void* out, void* ws, size_t ws_bytes, int32_t* err,
+                           void* stream);
+size_t csa_sparse_attn_workspace_bytes(const csa_params* params, int32_t T);
+
+/* ------------------------------------------------------------------------
+ * hca_dense_attn  [PACMAN 3.2; kwkr 3.2, 3.3; WeChat 1.1]
+ *
+ * As csa_sparse_attn with J = every visible cache entry 0 .. n_t-1
+ * (n_t = floor((t+1)/m)) followed by the window.  n_max is a host upper
+ * bound on n_t (<= cache.cap).
+ * ---------------------------------------------------------------------- */
+csa_status hca_dense_attn(const csa_params* params, const void* q,
+                          csa_kv cache, csa_kv win, const float* sink,
+                          const int32_t* q_pos0, int32_t T, int32_t n_max,
+                          void* out, void* ws, size_t ws_bytes, int32_t* err,
+                          void* stream);
+size_t hca_dense_attn_workspace_bytes(const csa_params* params, int32_t T,
+                                      int32_t n_max);
+
+/* Human-readable name of a csa_status. */
+const char* csa_status_string(csa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H_ */

@@ -1,0 +1,99 @@
+// Device helpers shared by the CSA/HCA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csa.h"
+
+namespace csa {
+
+constexpr float kE4M3Max = 448.0f;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t v) {
+  return __uint_as_float((v & 0xFFFFu) << 16);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code & 0xFF), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// round to nearest even, saturating to +-448
+__device__ __forceinline__ uint32_t f32_to_e4m3_sat(float f) {
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3));
+}
+
+// E2M1 nibble -> float, assembled from the bit fields (OCP MX: bias 1, one
+// mantissa bit, exponent field 0 is the subnormal 0 / 0.5).
+__device__ __forceinline__ float e2m1_to_f32(uint32_t n) {
+  uint32_t e = (n >> 1) & 3u, mt = n & 1u, s = (n >> 3) & 1u;
+  uint32_t bits = e ? (((e + 126u) << 23) | (mt << 22)) : (mt ? (126u << 23) : 0u);
+  return __uint_as_float(bits | (s << 31));
+}
+
+// UE8M0 scale byte -> 2^(E-127); 0xFF -> NaN
+__device__ __forceinline__ float ue8m0_to_f32(uint32_t e) {
+  e &= 0xFFu;
+  if (e == 0xFFu) return __uint_as_float(0x7FC00000u);
+  if (e == 0u) return __uint_as_float(0x00400000u);
+  return __uint_as_float(e << 23);
+}
+
+__device__ __forceinline__ void raise_err(int32_t* err, int32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide reductions; `red` holds >= 32 floats.  All threads must call.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float r = (lane < nw) ? red[lane] : 0.f;
+  r = warp_sum(r);
+  return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float r = (lane < nw) ? red[lane] : -INFINITY;
+  r = warp_max(r);
+  return r;
+}
+
+// RoPE angle of pair j (of r/2) at position pos, in double precision so that
+// positions up to 2^20 and beyond keep a small absolute angle error.
+__device__ __forceinline__ void rope_cos_sin(double pos, int j, int r, double theta, float* c, float* s) {
+  double freq = pow(theta, -2.0 * (double)j / (double)r);
+  double sn, cs;
+  sincos(pos * freq, &sn, &cs);
+  *c = (float)cs;
+  *s = (float)sn;
+}
+
+}  // namespace csa

@@ -1,0 +1,180 @@
+// Gated two-stream token compressor (CSA m=4, HCA m=128) with RMSNorm,
+// partial RoPE and the mixed FP8/BF16 pack, one CTA per (entry, sequence).
+//
+// kwkr.cn notes 3.1 (two KV streams merged with softmax-normalised gate
+// weights, adjacent blocks overlap), 3.2 (HCA: 128 tokens per entry);
+// Qiaomu blog 混合注意力机制 (entries normalised, RoPE on part of the dims);
+// WeChat 未来科技 1.1 (RoPE on the last 64 dims; RoPE dims BF16, others FP8).
+//
+// Thread layout: the d dims are split into d/4 quads; G = blockDim/(d/4)
+// thread groups each sum a strided subset of the 2m token rows, then the
+// groups' partial sums are reduced in shared memory.  Every stream row is
+// read once with 8-byte (bf16) or 16-byte (f32) coalesced loads.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+template <bool kF32>
+__device__ __forceinline__ void load4(const void* base, int64_t off, float v[4]) {
+  if (kF32) {
+    float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    uint2 x = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + off);
+    v[0] = bf16_bits_to_f32(x.x); v[1] = bf16_bits_to_f32(x.x >> 16);
+    v[2] = bf16_bits_to_f32(x.y); v[3] = bf16_bits_to_f32(x.y >> 16);
+  }
+}
+
+template <bool kF32, bool kKvF32>
+__global__ void __launch_bounds__(1024) compress_kernel(
+    const csa_params p, const void* __restrict__ a, const void* __restrict__ b,
+    const float* __restrict__ gate, int64_t S, const int32_t* __restrict__ tok_base,
+    const int32_t* __restrict__ e_begin, const int32_t* __restrict__ e_end,
+    const float* __restrict__ norm_w, uint8_t* __restrict__ rows, float* __restrict__ scale,
+    int64_t cap, int32_t* __restrict__ out_pos, int32_t* __restrict__ err) {
+  extern __shared__ float smem[];
+  const int m = p.m, d = p.d, r = p.r;
+  const int quads = d >> 2;
+  const int G = blockDim.x / quads;  // token groups
+  float* w = smem;                    // [2m] gate weights
+  float* part = smem + 2 * m;         // [G][d] partial sums
+  __shared__ float red[32];
+
+  const int bs = blockIdx.y;
+  const int64_t e = (int64_t)e_begin[bs] + blockIdx.x;
+  if (e >= e_end[bs]) return;
+  const int64_t base = tok_base[bs];
+  const int64_t ia0 = (int64_t)m * e - base;
+  const int nb = e > 0 ? m : 0;
+  const int64_t ib0 = (int64_t)m * (e - 1) - base;
+  if (ia0 < 0 || ia0 + m > S || (nb && ib0 < 0) || e >= cap) {
+    if (threadIdx.x == 0) raise_err(err, CSA_DEV_ERR_RANGE);
+    return;
+  }
+  const int n = m + nb;
+  const int64_t row0 = (int64_t)bs * S;
+
+  // 1. softmax over the union of both streams' logits
+  float lmax = -INFINITY;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    float g = i < m ? gate[(row0 + ia0 + i) * 2 + 0] : gate[(row0 + ib0 + (i - m)) * 2 + 1];
+    w[i] = g;
+    lmax = fmaxf(lmax, g);
+  }
+  const float gmax = block_max(lmax, red);
+  float lsum = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    float ex = expf(w[i] - gmax);
+    w[i] = ex;
+    lsum += ex;
+  }
+  const float inv = 1.f / block_sum(lsum, red);  // block_sum syncs: w[] is visible
+
+  // 2. weighted merge: group g sums rows i = g, g+G, ...
+  const int q = threadIdx.x % quads, g = threadIdx.x / quads;
+  const int d0 = q * 4;
+  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  if (g < G) {
+#pragma unroll 4
+    for (int i = g; i < n; i += G) {
+      float v[4];
+      if (i < m)
+        load4<kF32>(a, (row0 + ia0 + i) * d + d0, v);
+      else
+        load4<kF32>(b, (row0 + ib0 + (i - m)) * d + d0, v);
+      const float wi = w[i] * inv;
+      x[0] = fmaf(wi, v[0], x[0]); x[1] = fmaf(wi, v[1], x[1]);
+      x[2] = fmaf(wi, v[2], x[2]); x[3] = fmaf(wi, v[3], x[3]);
+    }
+    *reinterpret_cast<float4*>(part + g * d + d0) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+  __syncthreads();
+  const bool owner = threadIdx.x < quads;  // group 0 finishes the entry
+  float y[4] = {0.f, 0.f, 0.f, 0.f};
+  if (owner) {
+    for (int gg = 0; gg < G; ++gg) {
+      float4 t = *reinterpret_cast<const float4*>(part + gg * d + d0);
+      y[0] += t.x; y[1] += t.y; y[2] += t.z; y[3] += t.w;
+    }
+  }
+  // 3. RMSNorm
+  float ss = owner ? (y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3]) : 0.f;
+  const float tot = block_sum(ss, red);
+  const float rs = 1.f / sqrtf(tot / (float)d + p.eps);
+  if (!owner) return;  // no block-wide barrier below this point except via red in FP8 path
+#pragma unroll
+  for (int k = 0; k < 4; ++k) y[k] *= rs * (norm_w ? norm_w[d0 + k] : 1.f);
+  // 4. RoPE on the last r dims, pairs (d-r+2j, d-r+2j+1), angle (m*e)*theta^(-2j/r)
+  if (d0 >= d - r) {
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const int j = (d0 + 2 * pr - (d - r)) >> 1;
+      float c, s;
+      rope_cos_sin((double)(m * e), j, r, (double)p.rope_theta, &c, &s);
+      const float x0 = y[2 * pr], x1 = y[2 * pr + 1];
+      y[2 * pr] = x0 * c - x1 * s;
+      y[2 * pr + 1] = x0 * s + x1 * c;
+    }
+  }
+  const int64_t slot = (int64_t)bs * cap + e;
+  if (out_pos && threadIdx.x == 0) out_pos[slot] = (int32_t)(m * e);
+  if (kKvF32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(rows) + slot * d + d0) =
+        make_float4(y[0], y[1], y[2], y[3]);
+    return;
+  }
+  // 5. pack: E4M3 codes of x/scale (scale = amax/448 over the non-RoPE
+  //    dims) and BF16 RoPE dims.  Only the `quads` owner threads (a whole
+  //    number of warps when quads % 32 == 0) take part from here on.
+  float am = 0.f;
+  if (d0 < d - r) am = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+  am = warp_max(am);
+  __shared__ float wmax[32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) wmax[wid] = am;
+  asm volatile("bar.sync 1, %0;" ::"r"(quads));  // named barrier over the owners
+  float amax = 0.f;
+  for (int i = 0; i < (quads + 31) / 32; ++i) amax = fmaxf(amax, wmax[i]);
+  const float sc = amax > 0.f ? amax / kE4M3Max : 1.f;
+  const int64_t rb = (int64_t)(d + r);
+  uint8_t* row = rows + slot * rb;
+  if (d0 < d - r) {
+    uint32_t c = f32_to_e4m3_sat(y[0] / sc) | (f32_to_e4m3_sat(y[1] / sc) << 8) |
+                 (f32_to_e4m3_sat(y[2] / sc) << 16) | (f32_to_e4m3_sat(y[3] / sc) << 24);
+    *reinterpret_cast<uint32_t*>(row + d0) = c;
+  } else {
+    uint2 v;
+    v.x = (uint32_t)f32_to_bf16_bits(y[0]) | ((uint32_t)f32_to_bf16_bits(y[1]) << 16);
+    v.y = (uint32_t)f32_to_bf16_bits(y[2]) | ((uint32_t)f32_to_bf16_bits(y[3]) << 16);
+    *reinterpret_cast<uint2*>(row + (d - r) + 2 * (d0 - (d - r))) = v;
+  }
+  if (threadIdx.x == 0) scale[slot] = sc;
+}
+
+cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, const float* gate,
+                            int64_t S, const int32_t* tok_base, const int32_t* e_begin,
+                            const int32_t* e_end, int32_t max_entries, const float* norm_w,
+                            const csa_kv& out, int32_t* out_pos, int32_t* err, cudaStream_t st) {
+  const int quads = p.d / 4;
+  // more token groups for long blocks (HCA): more loads in flight per entry
+  int threads = p.m >= 64 ? 1024 : 256;
+  if (threads < quads) threads = quads;
+  const int G = threads / quads;
+  const size_t smem = (size_t)(2 * p.m + G * p.d) * sizeof(float);
+  dim3 grid(max_entries, p.B);
+  const bool f32 = p.act_fmt == CSA_ACT_F32, kv32 = p.kv_fmt == CSA_KV_F32;
+  auto* rows = reinterpret_cast<uint8_t*>(out.rows);
+  if (f32 && kv32)
+    compress_kernel<true, true><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
+  else if (f32)
+    compress_kernel<true, false><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
+  else if (kv32)
+    compress_kernel<false, true><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
+  else
+    compress_kernel<false, false><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

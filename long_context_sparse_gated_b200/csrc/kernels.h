@@ -1,0 +1,32 @@
+// Internal launchers of libcsa (not part of the public ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "csa.h"
+
+namespace csa {
+
+cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, const float* gate,
+                            int64_t S, const int32_t* tok_base, const int32_t* e_begin,
+                            const int32_t* e_end, int32_t max_entries, const float* norm_w,
+                            const csa_kv& out, int32_t* out_pos, int32_t* err, cudaStream_t st);
+
+cudaError_t launch_index_scores(const csa_params& p, const void* q_idx, const uint8_t* q_sf,
+                                const float* w, const void* k_idx, const uint8_t* k_sf,
+                                int64_t k_cap, const int32_t* q_pos0, int T, float* scores,
+                                int n_max, int32_t* err, cudaStream_t st);
+
+cudaError_t launch_topk(const csa_params& p, const float* scores, int n_max, const int32_t* q_pos0,
+                        int T, int64_t k_cap, int32_t* out_idx, cudaStream_t st);
+
+size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel);
+
+cudaError_t launch_attn(const csa_params& p, const void* q, const csa_kv& cache, const int32_t* idx,
+                        const csa_kv& win, const float* sink, const int32_t* q_pos0, int T,
+                        int n_sel, bool dense, void* out, float* ws, int32_t* err,
+                        cudaStream_t st);
+
+}  // namespace csa
