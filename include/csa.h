@@ -74,6 +74,7 @@ typedef int32_t csa_status;
 /* ---- device anomaly bits, OR-ed into *err ------------------------------ */
 #define CSA_DEV_ERR_INDEX 1  /* a top-k index >= visible entries or < -1   */
 #define CSA_DEV_ERR_RANGE 2  /* a token/entry range outside its buffer     */
+#define CSA_DEV_ERR_TIMEOUT 4 /* a bounded on-chip wait gave up (no hang)  */
 
 /* ---- formats ------------------------------------------------------------ */
 #define CSA_KV_F32 0

@@ -2,6 +2,7 @@
 // allocates, synchronises or keeps state; every call only enqueues kernels
 // on the caller's stream.
 #include <cuda_runtime.h>
+#include <stdlib.h>
 
 #include "csa.h"
 #include "kernels.h"
@@ -39,6 +40,13 @@ csa_status check_kv(const csa_params* p, const csa_kv& kv) {
     if (!aligned16(kv.scale)) return CSA_ERR_ALIGN;
   }
   return CSA_OK;
+}
+
+// CSA_INDEXER=simt selects the CUDA-core indexer instead of the tensor-core
+// one (a diagnostic switch: both compute the same scores).
+bool simt_indexer_requested() {
+  const char* v = getenv("CSA_INDEXER");
+  return v && v[0] == 's';
 }
 
 csa_status launched(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_LAUNCH; }
@@ -117,8 +125,13 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* scores = reinterpret_cast<float*>(ws);
   if (n_max > 0) {
-    cudaError_t e = csa::launch_index_scores(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0,
-                                             T, scores, n_max, err, st);
+    cudaError_t e;
+    if (csa::index_scores_tc_supported(*p, k_cap, q_idx, q_idx_sf, k_idx, k_idx_sf) && !simt_indexer_requested())
+      e = csa::launch_index_scores_tc(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0, T, scores, n_max,
+                                      err, st);
+    else
+      e = csa::launch_index_scores(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0, T, scores, n_max,
+                                   err, st);
     if (e != cudaSuccess) return CSA_ERR_LAUNCH;
   }
   return launched(csa::launch_topk(*p, scores, n_max, q_pos0, T, k_cap, out_idx, st));

@@ -1,0 +1,323 @@
+// Lightning Indexer scores on the 5th-generation tensor cores (sm_100a).
+//
+// Qiaomu blog 混合注意力机制 / FP4量化感知训练 and kwkr.cn notes 3.4, 4.4: the
+// indexer QK runs in FP4.  Here it runs as a block-scaled MXFP4 MMA
+// (tcgen05.mma kind::mxf4, E2M1 operands, one UE8M0 scale per 32 elements):
+//
+//   D[s, h] = sum_c k[s, c] * q[h, c]       (A = 128 index keys, K-major,
+//                                            B = the query's 64 heads)
+//   I(t, s) = sum_h w_h * max(D[s, h], 0)   (epilogue, fp32, h = 0..63)
+//
+// Persistent, warp-specialised CTA (one per SM), 192 threads:
+//   warp 0     TMA producer: per tile the 128x64 B key block (64B swizzle),
+//              the 64x64 B query block, and the raw scale-factor words of
+//              both, into an kStages-deep shared-memory ring
+//   warp 1     MMA issuer: permutes the scale factors into the 32x16 B
+//              layout tcgen05.cp expects, copies them to TMEM and issues two
+//              K=64 MMAs into one of two TMEM accumulators
+//   warps 2-5  epilogue: tcgen05.ld of the 64 head columns of one entry per
+//              thread, ReLU, weighted head sum, coalesced fp32 store
+// Each CTA walks a contiguous range of (query, 128-entry block) tiles, so the
+// key stream it reads is sequential.  Tiles past a query's n_t are skipped.
+//
+// Numerics: with MXFP4 inputs whose per-32 scales are >= 2^-2 and dyadic
+// head weights, every partial sum is exactly representable in fp32 (the
+// workloads check a bound), so the scores equal the exact scores.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kStages = 8;
+constexpr int kTileM = 128;   // entries per tile
+constexpr int kHeads = 64;    // index heads (N)
+constexpr int kRowBytes = 64; // 128 E2M1 values
+constexpr int kKeyBytes = kTileM * kRowBytes;   // 8192
+constexpr int kQBytes = kHeads * kRowBytes;     // 4096
+constexpr int kSfkBytes = kTileM * 4;           // 512 (4 UE8M0 per row)
+constexpr int kSfqBytes = kHeads * 4;           // 256
+constexpr uint32_t kTxBytes = kKeyBytes + kQBytes + kSfkBytes + kSfqBytes;
+
+struct __align__(1024) Stage {
+  uint8_t key[kKeyBytes];   // 1024-aligned (64B-swizzle atoms are 512 B)
+  uint8_t q[kQBytes];
+  uint32_t sfk_raw[kTileM];
+  uint32_t sfq_raw[kHeads];
+  uint32_t sfk[kTileM];     // permuted for tcgen05.cp (32 lines x 16 B)
+  uint32_t sfq[kTileM];     // rows 64..127 zero
+};
+
+struct Smem {
+  Stage st[kStages];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr uint32_t kTmemCols = 256;  // 2 x 64 accumulator columns + 2 x 8 scale columns
+
+__device__ __forceinline__ int visible(const int32_t* q_pos0, int T, int m, int qi, int n_max) {
+  const int bs = qi / T, tq = qi % T;
+  const int64_t t = (int64_t)q_pos0[bs] + tq;
+  int64_t n = (t + 1) / m;
+  return (int)(n < n_max ? n : n_max);
+}
+
+__global__ void __launch_bounds__(192, 1) index_scores_tc(
+    const __grid_constant__ CUtensorMap tm_key, const __grid_constant__ CUtensorMap tm_q,
+    const __grid_constant__ CUtensorMap tm_sfk, const __grid_constant__ CUtensorMap tm_sfq,
+    const float* __restrict__ w, const int32_t* __restrict__ q_pos0, int T, int m, int64_t k_cap,
+    int n_queries, int n_max, float* __restrict__ scores, int32_t* __restrict__ err) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tpq = (n_max + kTileM - 1) / kTileM;  // tiles per query
+  const int64_t n_tiles = (int64_t)n_queries * tpq;
+  const int64_t t_begin = n_tiles * blockIdx.x / gridDim.x;
+  const int64_t t_end = n_tiles * (blockIdx.x + 1) / gridDim.x;
+  volatile int* abort = &S.abort;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      sm100::mbar_init(&S.full[i], 1);
+      sm100::mbar_init(&S.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&S.tfull[i], 1);
+      sm100::mbar_init(&S.tempty[i], 4);
+    }
+    S.abort = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(&S.tmem_base, kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  // zero the padding rows of the permuted query scale blocks once
+  for (int i = threadIdx.x; i < kStages * kTileM; i += blockDim.x) S.st[i / kTileM].sfq[i % kTileM] = 0;
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      sm100::prefetch_tmap(&tm_key);
+      sm100::prefetch_tmap(&tm_q);
+      sm100::prefetch_tmap(&tm_sfk);
+      sm100::prefetch_tmap(&tm_sfq);
+      uint32_t it = 0;
+      for (int64_t t = t_begin; t < t_end; ++t) {
+        const int qi = (int)(t / tpq), j = (int)(t % tpq);
+        if (j * kTileM >= visible(q_pos0, T, m, qi, n_max)) continue;
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!sm100::mbar_wait(&S.empty[s], ph ^ 1, abort)) break;
+        Stage& st = S.st[s];
+        sm100::mbar_arrive_expect_tx(&S.full[s], kTxBytes);
+        const int bs = qi / T;
+        const int32_t row = (int32_t)((int64_t)bs * k_cap + (int64_t)j * kTileM);
+        sm100::tma_load_2d(st.key, &tm_key, &S.full[s], 0, row);
+        sm100::tma_load_1d(st.sfk_raw, &tm_sfk, &S.full[s], row);
+        sm100::tma_load_2d(st.q, &tm_q, &S.full[s], 0, qi * kHeads);
+        sm100::tma_load_1d(st.sfq_raw, &tm_sfq, &S.full[s], qi * kHeads);
+        ++it;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    uint32_t it = 0;
+    for (int64_t t = t_begin; t < t_end; ++t) {
+      const int qi = (int)(t / tpq), j = (int)(t % tpq);
+      if (j * kTileM >= visible(q_pos0, T, m, qi, n_max)) continue;
+      const int s = it % kStages;
+      const uint32_t ph = (it / kStages) & 1;
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort)) break;
+      if (!sm100::mbar_wait(&S.full[s], ph, abort)) break;
+      sm100::tc_fence_after();
+      Stage& st = S.st[s];
+      // scale factors: row r's word goes to line r%32, slot r/32
+      {
+        uint4 v;
+        v.x = st.sfk_raw[lane];
+        v.y = st.sfk_raw[lane + 32];
+        v.z = st.sfk_raw[lane + 64];
+        v.w = st.sfk_raw[lane + 96];
+        reinterpret_cast<uint4*>(st.sfk)[lane] = v;
+        uint4 u;
+        u.x = st.sfq_raw[lane];
+        u.y = st.sfq_raw[lane + 32];
+        u.z = 0u;
+        u.w = 0u;
+        reinterpret_cast<uint4*>(st.sfq)[lane] = u;
+      }
+      sm100::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t d_col = tmem + acc * kHeads;
+        const uint32_t sfa_col = tmem + 128 + acc * 8;
+        const uint32_t sfb_col = sfa_col + 4;
+        sm100::tc_cp_32x128b_warpx4(sfa_col, sm100::smem_desc(sm100::smem_u32(st.sfk), 0, 128, 0));
+        sm100::tc_cp_32x128b_warpx4(sfb_col, sm100::smem_desc(sm100::smem_u32(st.sfq), 0, 128, 0));
+        const uint32_t ka = sm100::smem_u32(st.key), qa = sm100::smem_u32(st.q);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          // K elements [64kk, 64kk+64) = bytes [32kk, 32kk+32) of every row
+          const uint64_t adesc = sm100::smem_desc(ka + 32 * kk, 16, 512, 4);
+          const uint64_t bdesc = sm100::smem_desc(qa + 32 * kk, 16, 512, 4);
+          sm100::mma_mxf4(d_col, adesc, bdesc, sm100::idesc_mxf4(kTileM, kHeads, 2 * kk, 2 * kk), sfa_col,
+                          sfb_col, kk);
+        }
+        sm100::tc_commit(&S.empty[s]);
+        sm100::tc_commit(&S.tfull[acc]);
+      }
+      __syncwarp();
+      ++it;
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = quad * 32 + lane;
+    uint32_t it = 0;
+    for (int64_t t = t_begin; t < t_end; ++t) {
+      const int qi = (int)(t / tpq), j = (int)(t % tpq);
+      const int n_t = visible(q_pos0, T, m, qi, n_max);
+      if (j * kTileM >= n_t) continue;
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!sm100::mbar_wait(&S.tfull[acc], aph, abort)) break;
+      sm100::tc_fence_after();
+      uint32_t d[64];
+      const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + acc * kHeads;
+      sm100::tmem_ld_x16(base + 0, *reinterpret_cast<uint32_t(*)[16]>(d + 0));
+      sm100::tmem_ld_x16(base + 16, *reinterpret_cast<uint32_t(*)[16]>(d + 16));
+      sm100::tmem_ld_x16(base + 32, *reinterpret_cast<uint32_t(*)[16]>(d + 32));
+      sm100::tmem_ld_x16(base + 48, *reinterpret_cast<uint32_t(*)[16]>(d + 48));
+      sm100::tmem_ld_wait();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&S.tempty[acc]);
+      const float4* wq = reinterpret_cast<const float4*>(w + (int64_t)qi * kHeads);
+      float sc = 0.f;
+#pragma unroll
+      for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+        const float4 wv = __ldg(wq + h4);
+        sc = fmaf(wv.x, fmaxf(__uint_as_float(d[4 * h4 + 0]), 0.f), sc);
+        sc = fmaf(wv.y, fmaxf(__uint_as_float(d[4 * h4 + 1]), 0.f), sc);
+        sc = fmaf(wv.z, fmaxf(__uint_as_float(d[4 * h4 + 2]), 0.f), sc);
+        sc = fmaf(wv.w, fmaxf(__uint_as_float(d[4 * h4 + 3]), 0.f), sc);
+      }
+      const int s_idx = j * kTileM + row;
+      if (s_idx < n_t) scores[(int64_t)qi * n_max + s_idx] = sc;
+      ++it;
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (S.abort && threadIdx.x == 0) raise_err(err, CSA_DEV_ERR_TIMEOUT);
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- host side ----------------------------------------------------------------
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
+  EncodeFn f = encode_fn();
+  if (!f) return false;
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = f(map, dt, (cuuint32_t)rank, const_cast<void*>(base), (const cuuint64_t*)dims,
+                 (const cuuint64_t*)strides_bytes, (const cuuint32_t*)box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q_idx, const uint8_t* q_sf,
+                               const void* k_idx, const uint8_t* k_sf) {
+  if (p.idx_fmt != CSA_IDX_MXFP4 || p.n_idx_heads != kHeads || p.idx_dim != 128) return false;
+  if (k_cap % 4 != 0) return false;  // scale rows must start 16-byte aligned for TMA
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const uint8_t* q_sf, const float* w,
+                                   const void* k_idx, const uint8_t* k_sf, int64_t k_cap,
+                                   const int32_t* q_pos0, int T, float* scores, int n_max, int32_t* err,
+                                   cudaStream_t st) {
+  const int nq = p.B * T;
+  CUtensorMap tk, tq, tsk, tsq;
+  const uint64_t key_rows = (uint64_t)p.B * (uint64_t)k_cap;
+  {
+    uint64_t dims[2] = {kRowBytes, key_rows};
+    uint64_t str[1] = {kRowBytes};
+    uint32_t box[2] = {kRowBytes, kTileM};
+    if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t dims[2] = {kRowBytes, (uint64_t)nq * kHeads};
+    uint64_t str[1] = {kRowBytes};
+    uint32_t box[2] = {kRowBytes, kHeads};
+    if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t dims[1] = {key_rows};
+    uint64_t str[1] = {4};
+    uint32_t box[1] = {kTileM};
+    if (!make_map(&tsk, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, k_sf, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
+  {
+    uint64_t dims[1] = {(uint64_t)nq * kHeads};
+    uint64_t str[1] = {4};
+    uint32_t box[1] = {kHeads};
+    if (!make_map(&tsq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, q_sf, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tpq = (n_max + kTileM - 1) / kTileM;
+  const int64_t tiles = (int64_t)nq * tpq;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  if (grid == 0) return cudaSuccess;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(index_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  index_scores_tc<<<grid, 192, smem, st>>>(tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap, nq, n_max, scores, err);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -19,6 +19,14 @@ cudaError_t launch_index_scores(const csa_params& p, const void* q_idx, const ui
                                 int64_t k_cap, const int32_t* q_pos0, int T, float* scores,
                                 int n_max, int32_t* err, cudaStream_t st);
 
+bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q_idx, const uint8_t* q_sf,
+                               const void* k_idx, const uint8_t* k_sf);
+
+cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const uint8_t* q_sf, const float* w,
+                                   const void* k_idx, const uint8_t* k_sf, int64_t k_cap,
+                                   const int32_t* q_pos0, int T, float* scores, int n_max, int32_t* err,
+                                   cudaStream_t st);
+
 cudaError_t launch_topk(const csa_params& p, const float* scores, int n_max, const int32_t* q_pos0,
                         int T, int64_t k_cap, int32_t* out_idx, cudaStream_t st);
 
