@@ -221,6 +221,10 @@ size_t hca_dense_attn_workspace_bytes(const csa_params* params, int32_t T,
 /* Human-readable name of a csa_status. */
 const char* csa_status_string(csa_status s);
 
+/* The CUDA error string behind the last CSA_ERR_LAUNCH returned on the
+ * calling host thread ("no error" if there was none).  Diagnostic only. */
+const char* csa_last_error_string(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -37,12 +37,12 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID", -2: "CSA_ERR_UNSUPPORTED", -3: "CS
 
 EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_index_topk_workspace_bytes",
            "csa_sparse_attn", "csa_sparse_attn_workspace_bytes", "hca_dense_attn",
-           "hca_dense_attn_workspace_bytes", "csa_status_string"]
+           "hca_dense_attn_workspace_bytes", "csa_status_string", "csa_last_error_string"]
 
 
 class CsaError(RuntimeError):
-    def __init__(self, name, status):
-        super().__init__(f"{name} returned {STATUS.get(status, status)}")
+    def __init__(self, name, status, detail=""):
+        super().__init__(f"{name} returned {STATUS.get(status, status)}" + (f" ({detail})" if detail else ""))
         self.status = status
 
 
@@ -89,6 +89,8 @@ def lib(path: str | None = None):
     L.hca_dense_attn_workspace_bytes.restype = _SZ
     L.csa_status_string.argtypes = [_I32]
     L.csa_status_string.restype = ctypes.c_char_p
+    L.csa_last_error_string.argtypes = []
+    L.csa_last_error_string.restype = ctypes.c_char_p
     for n in ("csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn"):
         getattr(L, n).restype = _I32
     if path == LIB_PATH:
@@ -132,7 +134,8 @@ def _kv(rows, scale):
 
 def _check(name, st):
     if st != 0:
-        raise CsaError(name, st)
+        detail = lib().csa_last_error_string().decode() if st == -5 else ""
+        raise CsaError(name, st, detail)
 
 
 def csa_compress(params, a, b, gate, tok_base, e_begin, e_end, max_entries, out_rows, out_scale=None,

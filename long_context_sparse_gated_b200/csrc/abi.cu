@@ -49,7 +49,13 @@ bool simt_indexer_requested() {
   return v && v[0] == 's';
 }
 
-csa_status launched(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_LAUNCH; }
+thread_local const char* g_last_error = "no error";
+
+csa_status launched(cudaError_t e) {
+  if (e == cudaSuccess) return CSA_OK;
+  g_last_error = cudaGetErrorString(e);
+  return CSA_ERR_LAUNCH;
+}
 
 csa_status compress_impl(const csa_params* p, const void* a, const void* b, const float* gate,
                          int64_t S, const int32_t* tok_base, const int32_t* e_begin,
@@ -132,19 +138,19 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
     else
       e = csa::launch_index_scores(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0, T, scores, n_max,
                                    err, st);
-    if (e != cudaSuccess) return CSA_ERR_LAUNCH;
+    if (e != cudaSuccess) return launched(e);
   }
   return launched(csa::launch_topk(*p, scores, n_max, q_pos0, T, k_cap, out_idx, st));
 }
 
 size_t csa_sparse_attn_workspace_bytes(const csa_params* p, int32_t T) {
   if (!p || T < 1 || p->B < 1) return 0;
-  return csa::attn_workspace_bytes(*p, T, p->topk);
+  return csa::attn_workspace_bytes(*p, T, p->topk, false);
 }
 
 size_t hca_dense_attn_workspace_bytes(const csa_params* p, int32_t T, int32_t n_max) {
   if (!p || T < 1 || p->B < 1 || n_max < 0) return 0;
-  return csa::attn_workspace_bytes(*p, T, n_max);
+  return csa::attn_workspace_bytes(*p, T, n_max, true);
 }
 
 static csa_status attn_impl(const csa_params* p, const void* q, csa_kv cache, const int32_t* idx,
@@ -162,7 +168,7 @@ static csa_status attn_impl(const csa_params* p, const void* q, csa_kv cache, co
   if ((s = check_kv(p, cache)) != CSA_OK) return s;
   if ((s = check_kv(p, win)) != CSA_OK) return s;
   if (win.cap < p->window || win.cap < T) return CSA_ERR_INVALID;
-  const size_t need = csa::attn_workspace_bytes(*p, T, n_sel);
+  const size_t need = csa::attn_workspace_bytes(*p, T, n_sel, dense);
   if (ws_bytes < need || (need && !ws)) return CSA_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return CSA_ERR_ALIGN;
   return launched(csa::launch_attn(*p, q, cache, idx, win, sink, q_pos0, T, n_sel, dense, out,
@@ -184,6 +190,8 @@ csa_status hca_dense_attn(const csa_params* p, const void* q, csa_kv cache, csa_
   return attn_impl(p, q, cache, nullptr, win, sink, q_pos0, T, n_max, true, out, ws, ws_bytes, err,
                    stream);
 }
+
+const char* csa_last_error_string(void) { return g_last_error; }
 
 const char* csa_status_string(csa_status s) {
   switch (s) {

@@ -14,6 +14,8 @@
 // head group), runs an online softmax over 32-row tiles and either writes
 // the final output (single split) or an unnormalised partial (O, max,
 // sum) that attn_merge combines in split order.
+#include <stdlib.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -296,11 +298,27 @@ static cudaError_t launch_attn_t(const csa_params& p, const void* q, const csa_k
   kfn<<<grid, p.d / 2, smem, st>>>(p, q, rc, idx, rw, sink, q_pos0, T, n_sel, rps, n_splits, out, ws_o, ws_ml, err);
   e = cudaGetLastError();
   if (e != cudaSuccess || n_splits == 1) return e;
-  attn_merge<kActF32><<<dim3(p.B * T, p.n_heads), p.d / 2, 0, st>>>(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out);
+  return launch_attn_merge(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out, st);
+}
+
+cudaError_t launch_attn_merge(const csa_params& p, const float* ws_o, const float* ws_ml, int n_splits,
+                              const float* sink, const int32_t* q_pos0, int T, void* out, cudaStream_t st) {
+  if (p.act_fmt == CSA_ACT_F32)
+    attn_merge<true><<<dim3(p.B * T, p.n_heads), p.d / 2, 0, st>>>(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out);
+  else
+    attn_merge<false><<<dim3(p.B * T, p.n_heads), p.d / 2, 0, st>>>(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out);
   return cudaGetLastError();
 }
 
-size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel) {
+// CSA_ATTN=simt selects the CUDA-core attention (a diagnostic switch).
+static bool simt_attn_requested() {
+  const char* v = getenv("CSA_ATTN");
+  return v && v[0] == 's';
+}
+
+static bool use_tc(const csa_params& p) { return attn_tc_supported(p) && !simt_attn_requested(); }
+
+static size_t attn_simt_workspace_bytes(const csa_params& p, int T, int n_sel) {
   const int total = n_sel + p.window;
   const int rps = attn_rows_per_split(total, T);
   const int n_splits = (total + rps - 1) / rps;
@@ -308,10 +326,16 @@ size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel) {
   return (size_t)p.B * T * n_splits * p.n_heads * (p.d + 2) * sizeof(float);
 }
 
+size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense) {
+  if (use_tc(p)) return attn_tc_workspace_bytes(p, T, n_sel, dense);
+  return attn_simt_workspace_bytes(p, T, n_sel);
+}
+
 cudaError_t launch_attn(const csa_params& p, const void* q, const csa_kv& cache, const int32_t* idx,
                         const csa_kv& win, const float* sink, const int32_t* q_pos0, int T,
                         int n_sel, bool dense, void* out, float* ws, int32_t* err,
                         cudaStream_t st) {
+  if (use_tc(p)) return launch_attn_tc(p, q, cache, idx, win, sink, q_pos0, T, n_sel, dense, out, ws, err, st);
   const bool kv32 = p.kv_fmt == CSA_KV_F32, a32 = p.act_fmt == CSA_ACT_F32;
 #define CSA_ATTN_CASE(K, A, D) \
   if (kv32 == K && a32 == A && dense == D) \

@@ -30,7 +30,16 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
 cudaError_t launch_topk(const csa_params& p, const float* scores, int n_max, const int32_t* q_pos0,
                         int T, int64_t k_cap, int32_t* out_idx, cudaStream_t st);
 
-size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel);
+size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense);
+
+cudaError_t launch_attn_merge(const csa_params& p, const float* ws_o, const float* ws_ml, int n_splits,
+                              const float* sink, const int32_t* q_pos0, int T, void* out, cudaStream_t st);
+
+bool attn_tc_supported(const csa_params& p);
+size_t attn_tc_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense);
+cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cache, const int32_t* idx,
+                           const csa_kv& win, const float* sink, const int32_t* q_pos0, int T, int n_sel,
+                           bool dense, void* out, float* ws, int32_t* err, cudaStream_t st);
 
 cudaError_t launch_attn(const csa_params& p, const void* q, const csa_kv& cache, const int32_t* idx,
                         const csa_kv& win, const float* sink, const int32_t* q_pos0, int T,
