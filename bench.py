@@ -194,6 +194,8 @@ def main():
     ap.add_argument("--config", default="c1", choices=sorted(CONFIG_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="device copies rotated in the timed loop (0: enough to exceed 3x L2)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -225,6 +227,8 @@ def main():
     n_copies = max(1, int(np.ceil(3 * L2_BYTES / step_bytes)))
     if args.config == "c4":
         n_copies = 1  # prefill touches far more than L2 per step
+    if args.copies > 0:
+        n_copies = args.copies
     dws = [DeviceWorkload(w) for _ in range(n_copies)]
     p = w["params"]
     queries = p.B * w["T"]

@@ -77,9 +77,17 @@ csa_status compress_impl(const csa_params* p, const void* a, const void* b, cons
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// Index workspace: fp32 scores [B*T][ld] (ld = n_max rounded up to 32),
+// then, for decode-sized batches, a 4096-bin histogram per query.
 size_t scores_bytes(const csa_params* p, int32_t T, int32_t n_max) {
-  size_t b = (size_t)p->B * (size_t)T * (size_t)n_max * sizeof(float);
+  size_t b = (size_t)p->B * (size_t)T * (size_t)csa::topk_scores_ld(n_max) * sizeof(float);
   return (b + 255) & ~(size_t)255;
+}
+
+size_t index_ws_bytes(const csa_params* p, int32_t T, int32_t n_max) {
+  size_t b = scores_bytes(p, T, n_max);
+  if (csa::topk_use_hist(p->B * T)) b += csa::topk_hist_bytes(p->B * T);
+  return b;
 }
 
 }  // namespace
@@ -104,7 +112,7 @@ csa_status hca_compress(const csa_params* p, const void* a, const void* b, const
 
 size_t csa_index_topk_workspace_bytes(const csa_params* p, int32_t T, int32_t n_max) {
   if (!p || T < 1 || n_max < 0 || p->B < 1) return 0;
-  return scores_bytes(p, T, n_max);
+  return index_ws_bytes(p, T, n_max);
 }
 
 csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t* q_idx_sf,
@@ -125,22 +133,31 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
   for (const void* ptr : {q_idx, (const void*)w, k_idx, (const void*)q_pos0, (const void*)out_idx})
     if (!aligned16(ptr)) return CSA_ERR_ALIGN;
   if (mx && (!aligned16(q_idx_sf) || !aligned16(k_idx_sf))) return CSA_ERR_ALIGN;
-  const size_t need = scores_bytes(p, T, n_max);
+  const size_t need = index_ws_bytes(p, T, n_max);
   if (ws_bytes < need || (need && !ws)) return CSA_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return CSA_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* scores = reinterpret_cast<float*>(ws);
-  if (n_max > 0) {
-    cudaError_t e;
-    if (csa::index_scores_tc_supported(*p, k_cap, q_idx, q_idx_sf, k_idx, k_idx_sf) && !simt_indexer_requested())
-      e = csa::launch_index_scores_tc(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0, T, scores, n_max,
-                                      err, st);
-    else
-      e = csa::launch_index_scores(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0, T, scores, n_max,
-                                   err, st);
+  const int ld = csa::topk_scores_ld(n_max);
+  const bool tc = csa::index_scores_tc_supported(*p, k_cap, q_idx, q_idx_sf, k_idx, k_idx_sf) &&
+                  !simt_indexer_requested();
+  uint32_t* hist = nullptr;
+  if (tc && csa::topk_use_hist(p->B * T) && n_max > p->topk) {
+    hist = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + scores_bytes(p, T, n_max));
+    cudaError_t e = cudaMemsetAsync(hist, 0, csa::topk_hist_bytes(p->B * T), st);
     if (e != cudaSuccess) return launched(e);
   }
-  return launched(csa::launch_topk(*p, scores, n_max, q_pos0, T, k_cap, out_idx, st));
+  if (n_max > 0) {
+    cudaError_t e;
+    if (tc)
+      e = csa::launch_index_scores_tc(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0, T, scores, ld,
+                                      hist, n_max, err, st);
+    else
+      e = csa::launch_index_scores(*p, q_idx, q_idx_sf, w, k_idx, k_idx_sf, k_cap, q_pos0, T, scores, ld,
+                                   n_max, err, st);
+    if (e != cudaSuccess) return launched(e);
+  }
+  return launched(csa::launch_topk_select(*p, scores, ld, n_max, hist, q_pos0, T, out_idx, st));
 }
 
 size_t csa_sparse_attn_workspace_bytes(const csa_params* p, int32_t T) {

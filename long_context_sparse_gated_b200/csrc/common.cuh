@@ -86,6 +86,28 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
+// Order-preserving 32-bit key of an fp32 score: a larger score gives a
+// larger key, and -0 and +0 give the same key.
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) == 0) u = 0;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Warp-aggregated increment of hist[bin] for the lanes with `active` set.
+// Every lane of the warp must call it.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  const unsigned act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const unsigned peers = __match_any_sync(act, bin);
+  const int leader = __ffs(peers) - 1;
+  if ((int)(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
+// Bins of the per-query score histogram: the top 12 bits of the key.
+constexpr int kScoreHistBins = 4096;
+__device__ __forceinline__ uint32_t score_bin(float f) { return score_key(f) >> 20; }
+
 // RoPE angle of pair j (of r/2) at position pos, in double precision so that
 // positions up to 2^20 and beyond keep a small absolute angle error.
 __device__ __forceinline__ void rope_cos_sin(double pos, int j, int r, double theta, float* c, float* s) {

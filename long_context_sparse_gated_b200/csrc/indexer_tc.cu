@@ -16,7 +16,9 @@
 //              layout tcgen05.cp expects, copies them to TMEM and issues two
 //              K=64 MMAs into one of two TMEM accumulators
 //   warps 2-5  epilogue: tcgen05.ld of the 64 head columns of one entry per
-//              thread, ReLU, weighted head sum, coalesced fp32 store
+//              thread, ReLU, weighted head sum, coalesced fp32 store, and
+//              (optionally) the per-query histogram of the scores' top 12
+//              key bits that the top-k selector starts from
 // Each CTA walks a contiguous range of (query, 128-entry block) tiles, so the
 // key stream it reads is sequential.  Tiles past a query's n_t are skipped.
 //
@@ -75,7 +77,8 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
     const __grid_constant__ CUtensorMap tm_key, const __grid_constant__ CUtensorMap tm_q,
     const __grid_constant__ CUtensorMap tm_sfk, const __grid_constant__ CUtensorMap tm_sfq,
     const float* __restrict__ w, const int32_t* __restrict__ q_pos0, int T, int m, int64_t k_cap,
-    int n_queries, int n_max, float* __restrict__ scores, int32_t* __restrict__ err) {
+    int n_queries, int n_max, float* __restrict__ scores, int ld, uint32_t* __restrict__ hist,
+    int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -219,7 +222,8 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
         sc = fmaf(wv.w, fmaxf(__uint_as_float(d[4 * h4 + 3]), 0.f), sc);
       }
       const int s_idx = j * kTileM + row;
-      if (s_idx < n_t) scores[(int64_t)qi * n_max + s_idx] = sc;
+      if (s_idx < n_t) scores[(int64_t)qi * ld + s_idx] = sc;
+      if (hist) hist_add(hist + (int64_t)qi * kScoreHistBins, score_bin(sc), s_idx < n_t);
       ++it;
     }
   }
@@ -273,8 +277,8 @@ bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q
 
 cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const uint8_t* q_sf, const float* w,
                                    const void* k_idx, const uint8_t* k_sf, int64_t k_cap,
-                                   const int32_t* q_pos0, int T, float* scores, int n_max, int32_t* err,
-                                   cudaStream_t st) {
+                                   const int32_t* q_pos0, int T, float* scores, int ld, uint32_t* hist,
+                                   int n_max, int32_t* err, cudaStream_t st) {
   const int nq = p.B * T;
   CUtensorMap tk, tq, tsk, tsq;
   const uint64_t key_rows = (uint64_t)p.B * (uint64_t)k_cap;
@@ -316,7 +320,8 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(index_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  index_scores_tc<<<grid, 192, smem, st>>>(tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap, nq, n_max, scores, err);
+  index_scores_tc<<<grid, 192, smem, st>>>(tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap, nq, n_max, scores, ld,
+                                           hist, err);
   return cudaGetLastError();
 }
 

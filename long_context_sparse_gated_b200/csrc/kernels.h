@@ -17,18 +17,22 @@ cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, c
 cudaError_t launch_index_scores(const csa_params& p, const void* q_idx, const uint8_t* q_sf,
                                 const float* w, const void* k_idx, const uint8_t* k_sf,
                                 int64_t k_cap, const int32_t* q_pos0, int T, float* scores,
-                                int n_max, int32_t* err, cudaStream_t st);
+                                int ld, int n_max, int32_t* err, cudaStream_t st);
 
 bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q_idx, const uint8_t* q_sf,
                                const void* k_idx, const uint8_t* k_sf);
 
 cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const uint8_t* q_sf, const float* w,
                                    const void* k_idx, const uint8_t* k_sf, int64_t k_cap,
-                                   const int32_t* q_pos0, int T, float* scores, int n_max, int32_t* err,
-                                   cudaStream_t st);
+                                   const int32_t* q_pos0, int T, float* scores, int ld, uint32_t* hist,
+                                   int n_max, int32_t* err, cudaStream_t st);
 
-cudaError_t launch_topk(const csa_params& p, const float* scores, int n_max, const int32_t* q_pos0,
-                        int T, int64_t k_cap, int32_t* out_idx, cudaStream_t st);
+size_t topk_hist_bytes(int queries);
+bool topk_use_hist(int queries);
+int topk_scores_ld(int n_max);
+cudaError_t launch_topk_select(const csa_params& p, const float* scores, int ld, int n_max,
+                               const uint32_t* hist, const int32_t* q_pos0, int T, int32_t* out_idx,
+                               cudaStream_t st);
 
 size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense);
 

@@ -76,6 +76,6 @@ def test_host_validation_codes():
     assert r["n_max_gt_cap"] == -1
     assert r["null_sink"] == -1
     assert r["small_window"] == -1
-    assert r["ws_bytes"] == 2 * 32768 * 4
+    assert r["ws_bytes"] == 2 * 32768 * 4 + 2 * 4096 * 4  # scores + per-query histograms
     assert r["attn_ws"] > 0
     assert r["name"] == "CSA_ERR_WORKSPACE"

@@ -27,8 +27,11 @@ def _lib():
 
 
 def _scores(dw):
-    n = dw.p.B * dw.T * dw.n_max
-    return dw.ws_idx.view(torch.float32)[:n].view(dw.p.B * dw.T, dw.n_max).cpu().numpy()
+    """The fp32 scores the indexer leaves at the start of its workspace
+    (rows padded to a multiple of 32 entries)."""
+    ld = (dw.n_max + 31) // 32 * 32
+    n = dw.p.B * dw.T * ld
+    return dw.ws_idx.view(torch.float32)[:n].view(dw.p.B * dw.T, ld)[:, :dw.n_max].cpu().numpy()
 
 
 def _run_index(w, simt=False):
