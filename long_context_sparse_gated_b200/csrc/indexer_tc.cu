@@ -8,14 +8,15 @@
 //                                            B = the query's 64 heads)
 //   I(t, s) = sum_h w_h * max(D[s, h], 0)   (epilogue, fp32, h = 0..63)
 //
-// Persistent, warp-specialised CTA (one per SM), 192 threads:
+// Persistent, warp-specialised CTA (one per SM), 320 threads:
 //   warp 0     TMA producer: per tile the 128x64 B key block (64B swizzle),
 //              the 64x64 B query block, and the raw scale-factor words of
 //              both, into an kStages-deep shared-memory ring
 //   warp 1     MMA issuer: permutes the scale factors into the 32x16 B
 //              layout tcgen05.cp expects, copies them to TMEM and issues two
-//              K=64 MMAs into one of two TMEM accumulators
-//   warps 2-5  epilogue: tcgen05.ld of the 64 head columns of one entry per
+//              K=64 MMAs into one of four TMEM accumulators
+//   warps 2-9  two epilogue warpgroups taking alternate tiles (the epilogue
+//              is the longest stage): tcgen05.ld of the 64 head columns of one entry per
 //              thread, ReLU, weighted head sum, coalesced fp32 store, and
 //              (optionally) the per-query histogram of the scores' top 12
 //              key bits that the top-k selector starts from
@@ -54,17 +55,20 @@ struct __align__(1024) Stage {
   uint32_t sfq[kTileM];     // rows 64..127 zero
 };
 
+constexpr int kAcc = 4;         // TMEM accumulators (two per epilogue warpgroup)
+constexpr int kEpiGroups = 2;   // epilogue warpgroups, alternating tiles
+
 struct Smem {
   Stage st[kStages];
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[kAcc];
+  uint64_t tempty[kAcc];
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr uint32_t kTmemCols = 256;  // 2 x 64 accumulator columns + 2 x 8 scale columns
+constexpr uint32_t kTmemCols = 512;  // 4 x 64 accumulator columns + 4 x 8 scale columns
 
 __device__ __forceinline__ int visible(const int32_t* q_pos0, int T, int m, int qi, int n_max) {
   const int bs = qi / T, tq = qi % T;
@@ -73,7 +77,22 @@ __device__ __forceinline__ int visible(const int32_t* q_pos0, int T, int m, int 
   return (int)(n < n_max ? n : n_max);
 }
 
-__global__ void __launch_bounds__(192, 1) index_scores_tc(
+// visible() of the current query, re-read only when the query changes: the
+// single producer thread must not pay a global-load latency per tile.
+struct VisibleCache {
+  int qi = -1, n = 0;
+  __device__ __forceinline__ int get(const int32_t* q_pos0, int T, int m, int q, int n_max) {
+    if (q != qi) {
+      qi = q;
+      n = visible(q_pos0, T, m, q, n_max);
+    }
+    return n;
+  }
+};
+
+constexpr int kThreadsTc = 64 + 128 * kEpiGroups;  // producer, MMA, 2 epilogue warpgroups
+
+__global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     const __grid_constant__ CUtensorMap tm_key, const __grid_constant__ CUtensorMap tm_q,
     const __grid_constant__ CUtensorMap tm_sfk, const __grid_constant__ CUtensorMap tm_sfq,
     const float* __restrict__ w, const int32_t* __restrict__ q_pos0, int T, int m, int64_t k_cap,
@@ -93,7 +112,7 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
       sm100::mbar_init(&S.full[i], 1);
       sm100::mbar_init(&S.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAcc; ++i) {
       sm100::mbar_init(&S.tfull[i], 1);
       sm100::mbar_init(&S.tempty[i], 4);
     }
@@ -119,9 +138,10 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
       sm100::prefetch_tmap(&tm_sfk);
       sm100::prefetch_tmap(&tm_sfq);
       uint32_t it = 0;
+      VisibleCache vc;
       for (int64_t t = t_begin; t < t_end; ++t) {
         const int qi = (int)(t / tpq), j = (int)(t % tpq);
-        if (j * kTileM >= visible(q_pos0, T, m, qi, n_max)) continue;
+        if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!sm100::mbar_wait(&S.empty[s], ph ^ 1, abort)) break;
@@ -139,15 +159,18 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     uint32_t it = 0;
+    VisibleCache vc;
     for (int64_t t = t_begin; t < t_end; ++t) {
       const int qi = (int)(t / tpq), j = (int)(t % tpq);
-      if (j * kTileM >= visible(q_pos0, T, m, qi, n_max)) continue;
+      if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
       const int s = it % kStages;
       const uint32_t ph = (it / kStages) & 1;
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
-      if (!sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort)) break;
-      if (!sm100::mbar_wait(&S.full[s], ph, abort)) break;
+      const int acc = it % kAcc;
+      const uint32_t aph = (it / kAcc) & 1;
+      // one lane polls the barriers; the warp follows
+      int ok = 1;
+      if (lane == 0) ok = sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort) && sm100::mbar_wait(&S.full[s], ph, abort);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       sm100::tc_fence_after();
       Stage& st = S.st[s];
       // scale factors: row r's word goes to line r%32, slot r/32
@@ -169,7 +192,7 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
       __syncwarp();
       if (lane == 0) {
         const uint32_t d_col = tmem + acc * kHeads;
-        const uint32_t sfa_col = tmem + 128 + acc * 8;
+        const uint32_t sfa_col = tmem + kAcc * kHeads + acc * 8;
         const uint32_t sfb_col = sfa_col + 4;
         sm100::tc_cp_32x128b_warpx4(sfa_col, sm100::smem_desc(sm100::smem_u32(st.sfk), 0, 128, 0));
         sm100::tc_cp_32x128b_warpx4(sfb_col, sm100::smem_desc(sm100::smem_u32(st.sfq), 0, 128, 0));
@@ -189,17 +212,34 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
       ++it;
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    // ---------------- epilogue (warps 2..9: two warpgroups) ----------------
+    const int eg = (warp - 2) >> 2;  // warpgroup: tiles it with it % 2 == eg
+    const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
     uint32_t it = 0;
+    int wq = -1;
+    float wv[kHeads];
+    VisibleCache vc;
     for (int64_t t = t_begin; t < t_end; ++t) {
       const int qi = (int)(t / tpq), j = (int)(t % tpq);
-      const int n_t = visible(q_pos0, T, m, qi, n_max);
+      const int n_t = vc.get(q_pos0, T, m, qi, n_max);
       if (j * kTileM >= n_t) continue;
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
-      if (!sm100::mbar_wait(&S.tfull[acc], aph, abort)) break;
+      const uint32_t my = it++;
+      if ((int)(my % kEpiGroups) != eg) continue;
+      const int acc = my % kAcc;
+      const uint32_t aph = (my / kAcc) & 1;
+      if (qi != wq) {  // head weights of this tile's query, kept in registers
+        const float4* wp = reinterpret_cast<const float4*>(w + (int64_t)qi * kHeads);
+#pragma unroll
+        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+          const float4 v = __ldg(wp + h4);
+          wv[4 * h4] = v.x; wv[4 * h4 + 1] = v.y; wv[4 * h4 + 2] = v.z; wv[4 * h4 + 3] = v.w;
+        }
+        wq = qi;
+      }
+      int ok = 1;
+      if (lane == 0) ok = sm100::mbar_wait(&S.tfull[acc], aph, abort);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       sm100::tc_fence_after();
       uint32_t d[64];
       const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + acc * kHeads;
@@ -211,20 +251,12 @@ __global__ void __launch_bounds__(192, 1) index_scores_tc(
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&S.tempty[acc]);
-      const float4* wq = reinterpret_cast<const float4*>(w + (int64_t)qi * kHeads);
       float sc = 0.f;
 #pragma unroll
-      for (int h4 = 0; h4 < kHeads / 4; ++h4) {
-        const float4 wv = __ldg(wq + h4);
-        sc = fmaf(wv.x, fmaxf(__uint_as_float(d[4 * h4 + 0]), 0.f), sc);
-        sc = fmaf(wv.y, fmaxf(__uint_as_float(d[4 * h4 + 1]), 0.f), sc);
-        sc = fmaf(wv.z, fmaxf(__uint_as_float(d[4 * h4 + 2]), 0.f), sc);
-        sc = fmaf(wv.w, fmaxf(__uint_as_float(d[4 * h4 + 3]), 0.f), sc);
-      }
+      for (int h = 0; h < kHeads; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), sc);
       const int s_idx = j * kTileM + row;
       if (s_idx < n_t) scores[(int64_t)qi * ld + s_idx] = sc;
       if (hist) hist_add(hist + (int64_t)qi * kScoreHistBins, score_bin(sc), s_idx < n_t);
-      ++it;
     }
   }
 
@@ -320,7 +352,7 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(index_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  index_scores_tc<<<grid, 192, smem, st>>>(tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap, nq, n_max, scores, ld,
+  index_scores_tc<<<grid, kThreadsTc, smem, st>>>(tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap, nq, n_max, scores, ld,
                                            hist, err);
   return cudaGetLastError();
 }
