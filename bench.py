@@ -84,6 +84,19 @@ def algorithmic_bytes(w):
     return step, idx_call
 
 
+def launches_per_step(w):
+    """Kernels (and memset nodes) one step enqueues: compress, the indexer's
+    histogram memset + scorer + selector, attention (+ split merge)."""
+    p = w["params"]
+    n = 1 if w["S"] else 0
+    if p.k > 0:
+        n += 3 if w["T"] * p.B <= 4096 else 2
+        n += 2 if w["T"] <= 4 else 1
+    else:
+        n += 2 if w["T"] <= 4 else 1
+    return n
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
 
@@ -194,6 +207,7 @@ def main():
     ap.add_argument("--config", default="c1", choices=sorted(CONFIG_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every call from the host (no CUDA graphs)")
     ap.add_argument("--copies", type=int, default=0,
                     help="device copies rotated in the timed loop (0: enough to exceed 3x L2)")
     args = ap.parse_args()
@@ -254,13 +268,51 @@ def main():
         step(dws[i % n_copies])
     torch.cuda.synchronize()
 
+    # Each copy's step is captured as three CUDA graphs (compress, the
+    # dominant call, the rest) so that host launch cost does not starve the
+    # device; events between the replays time the dominant call.
+    graphs = []
+    if not args.no_graph:
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        for dw in dws:
+            parts = []
+            phases = [dw.compress, dw.index_topk, dw.sparse_attn] if p.k > 0 else [dw.compress, dw.dense_attn, None]
+            with torch.cuda.stream(cap):
+                for fn in phases:
+                    g = torch.cuda.CUDAGraph()
+                    if fn is not None:
+                        with torch.cuda.graph(g, stream=cap):
+                            fn()
+                    parts.append(g if fn is not None else None)
+            graphs.append(parts)
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+
+    def timed_step(i, ev=None):
+        if not graphs:
+            return step(dws[i % n_copies], ev)
+        g0, g1, g2 = graphs[i % n_copies]
+        g0.replay()
+        if ev is not None:
+            ev[0].record(stream)
+        g1.replay()
+        if ev is not None:
+            ev[1].record(stream)
+        if g2 is not None:
+            g2.replay()
+
+    for i in range(3):
+        timed_step(i)
+    torch.cuda.synchronize()
+
     sampler = ClockSampler(local)
     sampler.start()
     # keep the GPU busy while the sampler starts (untimed)
     t_end = time.perf_counter() + 0.5
     i = 0
     while time.perf_counter() < t_end:
-        step(dws[i % n_copies])
+        timed_step(i)
         i += 1
     torch.cuda.synchronize()
 
@@ -271,7 +323,7 @@ def main():
     torch.cuda.synchronize()
     t0.record(stream)
     for i in range(args.steps):
-        step(dws[i % n_copies], evs[i])
+        timed_step(i, evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -281,10 +333,11 @@ def main():
     # a little more load for the clock sampler, then stop it (untimed)
     t_end = time.perf_counter() + 0.3
     while time.perf_counter() < t_end:
-        step(dws[i % n_copies])
+        timed_step(i)
         i += 1
     torch.cuda.synchronize()
     clocks = sampler.stop()
+    del graphs
 
     # ---- end to end: per-step inputs from pinned host memory, results back --
     dw = dws[0]
@@ -340,7 +393,8 @@ def main():
         "config": {"workload": CONFIG_NAMES[args.config], "name": args.config, "batch": p.B,
                    "context": int(w["L"].max()), "queries_per_step": queries,
                    "l2": f"inputs larger than L2: {n_copies} device copies rotated, {n_copies * step_bytes / 2**20:.0f} MiB per cycle"},
-        "gpu_launches": args.steps * (5 if p.k > 0 else 3),
+        "gpu_launches": args.steps * launches_per_step(w),
+        "graphs": not args.no_graph,
         "roofline": {"bound": "hbm", "kernel": "csa_index_topk" if p.k > 0 else "hca_dense_attn",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": peak_kind, "traffic": None,
