@@ -218,6 +218,30 @@ csa_status hca_dense_attn(const csa_params* params, const void* q,
 size_t hca_dense_attn_workspace_bytes(const csa_params* params, int32_t T,
                                       int32_t n_max);
 
+/* ------------------------------------------------------------------------
+ * csa_index_topk_noalloc  (no counterpart in the DeepSeek-V4 write-ups: it
+ * is a deployment variant of csa_index_topk, not part of the method)
+ *
+ * csa_index_topk for callers that cannot allocate device memory -- e.g. a
+ * plugin handed only its inputs and outputs, or a loop that must not touch
+ * the allocator -- and so cannot provide the workspace.  Same arguments and
+ * results as csa_index_topk, minus ws/ws_bytes: the workspace is a static
+ * 16 MiB device array inside libcsa (held on every GPU that loads the
+ * library until the process exits).  Returns CSA_ERR_WORKSPACE, launching
+ * nothing, when csa_index_topk_workspace_bytes(params, T, n_max) exceeds
+ * 16 MiB.  It allocates nothing (no cudaMalloc/cudaFree, no allocating
+ * library call).  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  Every call shares the one array: calls
+ * whose work overlaps on the GPU race on it.
+ * ---------------------------------------------------------------------- */
+csa_status csa_index_topk_noalloc(const csa_params* params, const void* q_idx,
+                                  const uint8_t* q_idx_sf, const float* w,
+                                  const void* k_idx, const uint8_t* k_idx_sf,
+                                  int64_t k_cap, const int32_t* q_pos0, int32_t T,
+                                  int32_t n_max, int32_t* out_idx, int32_t* err,
+                                  void* stream);
+
 /* Human-readable name of a csa_status. */
 const char* csa_status_string(csa_status s);
 

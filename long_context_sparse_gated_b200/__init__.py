@@ -20,7 +20,7 @@ __all__ = [
     "CsaParams", "CsaKv", "CsaError", "lib", "make_params",
     "csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn",
     "csa_index_topk_workspace_bytes", "csa_sparse_attn_workspace_bytes",
-    "hca_dense_attn_workspace_bytes", "KV_F32", "KV_FP8_BF16", "IDX_F32", "IDX_MXFP4",
+    "hca_dense_attn_workspace_bytes", "csa_index_topk_noalloc", "KV_F32", "KV_FP8_BF16", "IDX_F32", "IDX_MXFP4",
     "ACT_F32", "ACT_BF16", "DEV_ERR_INDEX", "DEV_ERR_RANGE",
 ]
 
@@ -37,7 +37,8 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID", -2: "CSA_ERR_UNSUPPORTED", -3: "CS
 
 EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_index_topk_workspace_bytes",
            "csa_sparse_attn", "csa_sparse_attn_workspace_bytes", "hca_dense_attn",
-           "hca_dense_attn_workspace_bytes", "csa_status_string", "csa_last_error_string"]
+           "hca_dense_attn_workspace_bytes", "csa_status_string", "csa_last_error_string",
+           "csa_index_topk_noalloc"]
 
 
 class CsaError(RuntimeError):
@@ -81,6 +82,8 @@ def lib(path: str | None = None):
     L.csa_index_topk.argtypes = [_P, _V, _V, _V, _V, _V, _I64, _V, _I32, _I32, _V, _V, _SZ, _V, _V]
     L.csa_index_topk_workspace_bytes.argtypes = [_P, _I32, _I32]
     L.csa_index_topk_workspace_bytes.restype = _SZ
+    L.csa_index_topk_noalloc.argtypes = [_P, _V, _V, _V, _V, _V, _I64, _V, _I32, _I32, _V, _V, _V]
+    L.csa_index_topk_noalloc.restype = _I32
     L.csa_sparse_attn.argtypes = [_P, _V, CsaKv, _V, CsaKv, _V, _V, _I32, _V, _V, _SZ, _V, _V]
     L.csa_sparse_attn_workspace_bytes.argtypes = [_P, _I32]
     L.csa_sparse_attn_workspace_bytes.restype = _SZ
@@ -176,6 +179,17 @@ def csa_index_topk(params, q_idx, q_idx_sf, w, k_idx, k_idx_sf, q_pos0, T, n_max
                               _ptr(out_idx), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                               _ptr(err), _stream(stream))
     _check("csa_index_topk", st)
+
+
+def csa_index_topk_noalloc(params, q_idx, q_idx_sf, w, k_idx, k_idx_sf, q_pos0, T, n_max, out_idx,
+                           err=None, stream=None):
+    """csa_index_topk without a workspace argument, for callers that cannot
+    allocate device memory: the library's static 16 MiB device scratch is
+    used instead (shared by every call; overlapping calls race)."""
+    st = lib().csa_index_topk_noalloc(ctypes.byref(params), _ptr(q_idx), _ptr(q_idx_sf), _ptr(w),
+                                      _ptr(k_idx), _ptr(k_idx_sf), k_idx.shape[1], _ptr(q_pos0), int(T),
+                                      int(n_max), _ptr(out_idx), _ptr(err), _stream(stream))
+    _check("csa_index_topk_noalloc", st)
 
 
 def csa_sparse_attn(params, q, cache_rows, cache_scale, idx, win_rows, win_scale, sink, q_pos0, T, out,
