@@ -139,6 +139,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def recorded_traffic(key):
+    """DRAM bytes per launch of the dominant call from the committed ncu
+    capture (profiles/dram_traffic.json), or None when the kernels' sources
+    changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            e = json.load(f)[key]
+        h = hashlib.sha1()
+        for src in e["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        return int(e["bytes_per_launch"]) if h.hexdigest() == e["sources_sha1"] else None
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -397,7 +414,8 @@ def main():
         "graphs": not args.no_graph,
         "roofline": {"bound": "hbm", "kernel": "csa_index_topk" if p.k > 0 else "hca_dense_attn",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": peak_kind, "traffic": None,
+                     "peak_source": peak_kind,
+                     "traffic": recorded_traffic(f"csa_index_topk@{args.config}") if p.k > 0 else None,
                      "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean},
         "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
                           "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak},

@@ -6,8 +6,10 @@ Tolerances (stated once, used everywhere):
   * fp32 (config 0) outputs and compressed entries: max |diff| / max |oracle|
     <= 1e-5.
   * FP8 pack: E4M3 codes within one code step, per-row scale within 1e-6
-    relative, BF16 RoPE dims within one BF16 ulp (fp32 vs fp64 values may
-    straddle a rounding boundary).
+    relative (fp32 vs fp64 values may straddle a rounding boundary); BF16
+    RoPE dims within one BF16 ulp of the oracle's value plus 1e-6 absolute
+    (the kernel rotates in fp32: a rotated value near zero carries the
+    fp32 cancellation error of its unit-size inputs, ~1e-7).
   * Top-k sets: identical (they are unique: ties go to the lower index).
     On fp32 index data (config 0) a mismatch is accepted only where the
     oracle's k-th and (k+1)-th scores are within 1e-5 relative.
@@ -60,12 +62,11 @@ def check_fp8_rows(g_rows, g_scale, o_codes, o_scale, o_rbits, d, r, what=""):
                                rtol=1e-6, err_msg=f"{what}: scale")
     step = np.abs(_mag_index(g_codes) - _mag_index(o_codes))
     assert step.max() <= 1, f"{what}: E4M3 codes differ by {step.max()} steps"
-    gb = g_rbits.view(np.int16).astype(np.int64)
-    ob = np.asarray(o_rbits).view(np.int16).astype(np.int64)
-    # ordered integer line for sign-magnitude bf16
-    gl = np.where(gb < 0, -(gb & 0x7FFF), gb)
-    ol = np.where(ob < 0, -(ob & 0x7FFF), ob)
-    assert np.abs(gl - ol).max() <= 1, f"{what}: bf16 RoPE dims differ by > 1 ulp"
+    gv = bf16_to_f64(g_rbits)
+    ov = bf16_to_f64(o_rbits)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ov), 2.0 ** -126))) - 7)
+    bad = np.abs(gv - ov) > ulp + 1e-6
+    assert not bad.any(), f"{what}: bf16 RoPE dims differ: {gv[bad][:4]} vs {ov[bad][:4]}"
 
 
 def check_topk(g_idx, o_idx, o_scores=None, n_t=None, exact=True, what=""):
