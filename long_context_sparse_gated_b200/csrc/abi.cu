@@ -86,7 +86,7 @@ size_t scores_bytes(const csa_params* p, int32_t T, int32_t n_max) {
 
 size_t index_ws_bytes(const csa_params* p, int32_t T, int32_t n_max) {
   size_t b = scores_bytes(p, T, n_max);
-  if (csa::topk_use_hist(p->B * T)) b += csa::topk_hist_bytes(p->B * T);
+  if (csa::topk_use_hist(p->B * T)) b += csa::topk_hist_bytes(p->B * T) + csa::topk_cand_bytes(p->B * T, n_max);
   return b;
 }
 
@@ -157,7 +157,8 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
                                    n_max, err, st);
     if (e != cudaSuccess) return launched(e);
   }
-  return launched(csa::launch_topk_select(*p, scores, ld, n_max, hist, q_pos0, T, out_idx, st));
+  void* cand = hist ? reinterpret_cast<char*>(hist) + csa::topk_hist_bytes(p->B * T) : nullptr;
+  return launched(csa::launch_topk_select(*p, scores, ld, n_max, hist, q_pos0, T, out_idx, cand, st));
 }
 
 size_t csa_sparse_attn_workspace_bytes(const csa_params* p, int32_t T) {

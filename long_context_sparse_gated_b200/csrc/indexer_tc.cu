@@ -9,12 +9,14 @@
 //   I(t, s) = sum_h w_h * max(D[s, h], 0)   (epilogue, fp32, h = 0..63)
 //
 // Persistent, warp-specialised CTA (one per SM), 320 threads:
-//   warp 0     TMA producer: per tile the 128x64 B key block (64B swizzle),
-//              the 64x64 B query block, and the raw scale-factor words of
-//              both, into an kStages-deep shared-memory ring
-//   warp 1     MMA issuer: permutes the scale factors into the 32x16 B
-//              layout tcgen05.cp expects, copies them to TMEM and issues two
-//              K=64 MMAs into one of four TMEM accumulators
+//   warp 0     TMA producer: per tile the 128x64 B key block (64B swizzle,
+//              rows permuted by a 3-D view, see Stage) and its 512 scale
+//              bytes into a kStages-deep ring; per query (not per tile) the
+//              64x64 B query block and its scales into one of two slots
+//   warp 1     MMA issuer: per query, permutes the query scales into the
+//              32x16 B layout and copies them to TMEM; per tile, copies the
+//              key scales to TMEM (tcgen05.cp) and issues two K=64 MMAs into
+//              one of four TMEM accumulators
 //   warps 2-9  two epilogue warpgroups taking alternate tiles (the epilogue
 //              is the longest stage): tcgen05.ld of the 64 head columns of one entry per
 //              thread, ReLU, weighted head sum, coalesced fp32 store, and
@@ -36,7 +38,7 @@ namespace csa {
 
 namespace {
 
-constexpr int kStages = 8;
+constexpr int kStages = 12;
 constexpr int kTileM = 128;   // entries per tile
 constexpr int kHeads = 64;    // index heads (N)
 constexpr int kRowBytes = 64; // 128 E2M1 values
@@ -44,15 +46,23 @@ constexpr int kKeyBytes = kTileM * kRowBytes;   // 8192
 constexpr int kQBytes = kHeads * kRowBytes;     // 4096
 constexpr int kSfkBytes = kTileM * 4;           // 512 (4 UE8M0 per row)
 constexpr int kSfqBytes = kHeads * 4;           // 256
-constexpr uint32_t kTxBytes = kKeyBytes + kQBytes + kSfkBytes + kSfqBytes;
+constexpr uint32_t kStageTx = kKeyBytes + kSfkBytes;
+constexpr uint32_t kQueryTx = kQBytes + kSfqBytes;
 
+// A tile's 128 keys are loaded through a 3-D view of the key array, so that
+// MMA row 32q + i holds key 4i + q (q < 4, i < 32).  With that order the
+// keys' 512 contiguous scale bytes are already the 32-line x 16-byte block
+// tcgen05.cp expects (line i = scale words of MMA rows i, 32+i, 64+i, 96+i),
+// and no per-tile permutation is needed.
 struct __align__(1024) Stage {
   uint8_t key[kKeyBytes];   // 1024-aligned (64B-swizzle atoms are 512 B)
+  uint32_t sfk[kTileM];
+};
+
+struct __align__(1024) QuerySlot {
   uint8_t q[kQBytes];
-  uint32_t sfk_raw[kTileM];
   uint32_t sfq_raw[kHeads];
-  uint32_t sfk[kTileM];     // permuted for tcgen05.cp (32 lines x 16 B)
-  uint32_t sfq[kTileM];     // rows 64..127 zero
+  uint32_t sfq[kTileM];     // permuted for tcgen05.cp; rows 64..127 zero
 };
 
 constexpr int kAcc = 4;         // TMEM accumulators (two per epilogue warpgroup)
@@ -60,15 +70,22 @@ constexpr int kEpiGroups = 2;   // epilogue warpgroups, alternating tiles
 
 struct Smem {
   Stage st[kStages];
+  QuerySlot qs[2];
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  uint64_t qfull[2];
+  uint64_t qempty[2];
   uint64_t tfull[kAcc];
   uint64_t tempty[kAcc];
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr uint32_t kTmemCols = 512;  // 4 x 64 accumulator columns + 4 x 8 scale columns
+// TMEM columns: accumulators 0..255, key scales 256 + 4 acc, query scales
+// 272 + 4 slot.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfaCol = kAcc * kHeads;
+constexpr uint32_t kSfbCol = kSfaCol + 4 * kAcc;
 
 __device__ __forceinline__ int visible(const int32_t* q_pos0, int T, int m, int qi, int n_max) {
   const int bs = qi / T, tq = qi % T;
@@ -112,6 +129,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       sm100::mbar_init(&S.full[i], 1);
       sm100::mbar_init(&S.empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&S.qfull[i], 1);
+      sm100::mbar_init(&S.qempty[i], 1);
+    }
     for (int i = 0; i < kAcc; ++i) {
       sm100::mbar_init(&S.tfull[i], 1);
       sm100::mbar_init(&S.tempty[i], 4);
@@ -123,8 +144,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     sm100::tmem_alloc(&S.tmem_base, kTmemCols);
     sm100::tmem_relinquish();
   }
-  // zero the padding rows of the permuted query scale blocks once
-  for (int i = threadIdx.x; i < kStages * kTileM; i += blockDim.x) S.st[i / kTileM].sfq[i % kTileM] = 0;
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -137,32 +156,64 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       sm100::prefetch_tmap(&tm_q);
       sm100::prefetch_tmap(&tm_sfk);
       sm100::prefetch_tmap(&tm_sfq);
-      uint32_t it = 0;
+      uint32_t it = 0, nq = 0;
+      int cur_q = -1;
       VisibleCache vc;
       for (int64_t t = t_begin; t < t_end; ++t) {
         const int qi = (int)(t / tpq), j = (int)(t % tpq);
         if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
+        if (qi != cur_q) {  // the query's 64 heads, once per query
+          const int sl = nq & 1;
+          if (!sm100::mbar_wait(&S.qempty[sl], ((nq >> 1) & 1) ^ 1, abort)) break;
+          sm100::mbar_arrive_expect_tx(&S.qfull[sl], kQueryTx);
+          sm100::tma_load_2d(S.qs[sl].q, &tm_q, &S.qfull[sl], 0, qi * kHeads);
+          sm100::tma_load_1d(S.qs[sl].sfq_raw, &tm_sfq, &S.qfull[sl], qi * kHeads);
+          cur_q = qi;
+          ++nq;
+        }
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!sm100::mbar_wait(&S.empty[s], ph ^ 1, abort)) break;
         Stage& st = S.st[s];
-        sm100::mbar_arrive_expect_tx(&S.full[s], kTxBytes);
-        const int bs = qi / T;
-        const int32_t row = (int32_t)((int64_t)bs * k_cap + (int64_t)j * kTileM);
-        sm100::tma_load_2d(st.key, &tm_key, &S.full[s], 0, row);
-        sm100::tma_load_1d(st.sfk_raw, &tm_sfk, &S.full[s], row);
-        sm100::tma_load_2d(st.q, &tm_q, &S.full[s], 0, qi * kHeads);
-        sm100::tma_load_1d(st.sfq_raw, &tm_sfq, &S.full[s], qi * kHeads);
+        sm100::mbar_arrive_expect_tx(&S.full[s], kStageTx);
+        const int64_t row = (int64_t)(qi / T) * k_cap + (int64_t)j * kTileM;
+        sm100::tma_load_3d(st.key, &tm_key, &S.full[s], 0, (int32_t)(row / 4), 0);
+        sm100::tma_load_1d(st.sfk, &tm_sfk, &S.full[s], (int32_t)row);
         ++it;
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    uint32_t it = 0;
+    uint32_t it = 0, nq = 0;
+    int cur_q = -1, sl = 0;
     VisibleCache vc;
     for (int64_t t = t_begin; t < t_end; ++t) {
       const int qi = (int)(t / tpq), j = (int)(t % tpq);
       if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
+      if (qi != cur_q) {
+        // the previous query's slot is free once its MMAs complete
+        if (cur_q >= 0 && lane == 0) sm100::tc_commit(&S.qempty[sl]);
+        sl = nq & 1;
+        int ok = 1;
+        if (lane == 0) ok = sm100::mbar_wait(&S.qfull[sl], (nq >> 1) & 1, abort);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        // query scales: head h's word goes to line h%32, slot h/32
+        QuerySlot& qs = S.qs[sl];
+        uint4 u;
+        u.x = qs.sfq_raw[lane];
+        u.y = qs.sfq_raw[lane + 32];
+        u.z = 0u;
+        u.w = 0u;
+        reinterpret_cast<uint4*>(qs.sfq)[lane] = u;
+        sm100::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          sm100::tc_fence_after();
+          sm100::tc_cp_32x128b_warpx4(tmem + kSfbCol + 4 * sl, sm100::smem_desc(sm100::smem_u32(qs.sfq), 0, 128, 0));
+        }
+        cur_q = qi;
+        ++nq;
+      }
       const int s = it % kStages;
       const uint32_t ph = (it / kStages) & 1;
       const int acc = it % kAcc;
@@ -171,32 +222,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       int ok = 1;
       if (lane == 0) ok = sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort) && sm100::mbar_wait(&S.full[s], ph, abort);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      sm100::tc_fence_after();
-      Stage& st = S.st[s];
-      // scale factors: row r's word goes to line r%32, slot r/32
-      {
-        uint4 v;
-        v.x = st.sfk_raw[lane];
-        v.y = st.sfk_raw[lane + 32];
-        v.z = st.sfk_raw[lane + 64];
-        v.w = st.sfk_raw[lane + 96];
-        reinterpret_cast<uint4*>(st.sfk)[lane] = v;
-        uint4 u;
-        u.x = st.sfq_raw[lane];
-        u.y = st.sfq_raw[lane + 32];
-        u.z = 0u;
-        u.w = 0u;
-        reinterpret_cast<uint4*>(st.sfq)[lane] = u;
-      }
-      sm100::fence_proxy_async_smem();
-      __syncwarp();
       if (lane == 0) {
+        sm100::tc_fence_after();
+        Stage& st = S.st[s];
         const uint32_t d_col = tmem + acc * kHeads;
-        const uint32_t sfa_col = tmem + kAcc * kHeads + acc * 8;
-        const uint32_t sfb_col = sfa_col + 4;
+        const uint32_t sfa_col = tmem + kSfaCol + 4 * acc;
+        const uint32_t sfb_col = tmem + kSfbCol + 4 * sl;
         sm100::tc_cp_32x128b_warpx4(sfa_col, sm100::smem_desc(sm100::smem_u32(st.sfk), 0, 128, 0));
-        sm100::tc_cp_32x128b_warpx4(sfb_col, sm100::smem_desc(sm100::smem_u32(st.sfq), 0, 128, 0));
-        const uint32_t ka = sm100::smem_u32(st.key), qa = sm100::smem_u32(st.q);
+        const uint32_t ka = sm100::smem_u32(st.key), qa = sm100::smem_u32(S.qs[sl].q);
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
           // K elements [64kk, 64kk+64) = bytes [32kk, 32kk+32) of every row
@@ -215,7 +248,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     // ---------------- epilogue (warps 2..9: two warpgroups) ----------------
     const int eg = (warp - 2) >> 2;  // warpgroup: tiles it with it % 2 == eg
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;
+    // TMEM lane 32*quad + lane holds key 4*lane + quad of the tile
+    const int key_in_tile = 4 * lane + quad;
     uint32_t it = 0;
     int wq = -1;
     float wv[kHeads];
@@ -254,7 +288,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       float sc = 0.f;
 #pragma unroll
       for (int h = 0; h < kHeads; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), sc);
-      const int s_idx = j * kTileM + row;
+      const int s_idx = j * kTileM + key_in_tile;
       if (s_idx < n_t) scores[(int64_t)qi * ld + s_idx] = sc;
       if (hist) hist_add(hist + (int64_t)qi * kScoreHistBins, score_bin(sc), s_idx < n_t);
     }
@@ -291,7 +325,7 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* ba
               const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
   EncodeFn f = encode_fn();
   if (!f) return false;
-  cuuint32_t estr[2] = {1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = f(map, dt, (cuuint32_t)rank, const_cast<void*>(base), (const cuuint64_t*)dims,
                  (const cuuint64_t*)strides_bytes, (const cuuint32_t*)box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -315,10 +349,12 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
   CUtensorMap tk, tq, tsk, tsq;
   const uint64_t key_rows = (uint64_t)p.B * (uint64_t)k_cap;
   {
-    uint64_t dims[2] = {kRowBytes, key_rows};
-    uint64_t str[1] = {kRowBytes};
-    uint32_t box[2] = {kRowBytes, kTileM};
-    if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+    // (byte, i, q) -> byte + 256 i + 64 q: key row 4i + q lands in shared
+    // row 32q + (i mod 32)
+    uint64_t dims[3] = {kRowBytes, key_rows / 4, 4};
+    uint64_t str[2] = {4 * kRowBytes, kRowBytes};
+    uint32_t box[3] = {kRowBytes, kTileM / 4, 4};
+    if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
   {

@@ -30,9 +30,10 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
 size_t topk_hist_bytes(int queries);
 bool topk_use_hist(int queries);
 int topk_scores_ld(int n_max);
+size_t topk_cand_bytes(int queries, int n_max);
 cudaError_t launch_topk_select(const csa_params& p, const float* scores, int ld, int n_max,
                                const uint32_t* hist, const int32_t* q_pos0, int T, int32_t* out_idx,
-                               cudaStream_t st);
+                               void* cand, cudaStream_t st);
 
 size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense);
 
