@@ -287,21 +287,22 @@ def main():
 
     # Each copy's step is captured as three CUDA graphs (compress, the
     # dominant call, the rest) so that host launch cost does not starve the
-    # device; events between the replays time the dominant call.
+    # device; events between the replays time the dominant call alone.
     graphs = []
     if not args.no_graph:
         cap = torch.cuda.Stream()
         cap.wait_stream(stream)
         for dw in dws:
-            parts = []
             phases = [dw.compress, dw.index_topk, dw.sparse_attn] if p.k > 0 else [dw.compress, dw.dense_attn, None]
+            parts = []
             with torch.cuda.stream(cap):
                 for fn in phases:
-                    g = torch.cuda.CUDAGraph()
+                    g = None
                     if fn is not None:
+                        g = torch.cuda.CUDAGraph()
                         with torch.cuda.graph(g, stream=cap):
-                            fn()
-                    parts.append(g if fn is not None else None)
+                            fn(cap)
+                    parts.append(g)
             graphs.append(parts)
         stream.wait_stream(cap)
         torch.cuda.synchronize()
@@ -310,7 +311,8 @@ def main():
         if not graphs:
             return step(dws[i % n_copies], ev)
         g0, g1, g2 = graphs[i % n_copies]
-        g0.replay()
+        if g0 is not None:
+            g0.replay()
         if ev is not None:
             ev[0].record(stream)
         g1.replay()

@@ -25,8 +25,9 @@
 //   O^T       tcgen05.mma: O^T[c, h] += sum_j V'[j, c] P'[h, j]
 //             (A = V'^T, the same tile read MN-major; M = 128 dims x 4
 //             blocks, N = 64 heads, K = 128 rows) into TMEM
-//   epilogue  normalise with the sink term, inverse RoPE, BF16 store -- or
-//             write the unnormalised partial (O, m, l) for attn_merge.
+//   epilogue  normalise with the sink term, inverse RoPE, BF16 store -- or,
+//             with several splits, write the partial O/l (FP16) and (m, l)
+//             that attn_merge_f16 combines in split order.
 //
 // 8 warps (two per TMEM lane quadrant) gather, run the softmax and the
 // epilogue; thread 0 also issues the query TMA and the MMAs between block
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     const float* __restrict__ win_scale, int64_t win_cap, const int32_t* __restrict__ idx, int topk,
     const int32_t* __restrict__ q_pos0, int T, int m, int W, int n_sel, int n_heads, float tau,
     float theta, const float* __restrict__ sink, int rows_per_split, int n_splits, uint16_t* __restrict__ out,
-    float* __restrict__ ws_o, float* __restrict__ ws_ml, int32_t* __restrict__ err) {
+    __half* __restrict__ ws_o, float* __restrict__ ws_ml, int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& S = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -391,8 +392,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   sm100::tc_fence_after();
   __syncthreads();  // lh final; abort flag now uniform
   const bool ok = !S.abort;
+  const bool single = n_splits == 1;
   if (ok && n_tiles > 0) {
-    const bool single = n_splits == 1;
+    // single split: normalise with the sink term here; several splits: the
+    // partial normalised by its own sum, as FP16, plus (max, sum)
     float f[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
         const float den = expf(sg - ms) + (mh == -INFINITY ? 0.f : lh * expf(mh - ms));
         f[c] = (mh == -INFINITY || !(den > 0.f)) ? 0.f : expf(mh - ms) / den;
       } else {
-        f[c] = 1.f;
+        f[c] = lh > 0.f ? 1.f / lh : 0.f;
       }
     }
 #pragma unroll 1
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
             if (c_dim >= kNope) y = odd ? (pv * sn + y * cs) : (y * cs - pv * sn);
             out[((int64_t)qi * n_heads + h0 + h) * kD + c_dim] = f32_to_bf16_bits(y);
           } else {
-            ws_o[(((int64_t)qi * n_splits + split) * n_heads + h0 + h) * kD + c_dim] = y;
+            ws_o[(((int64_t)qi * n_splits + split) * n_heads + h0 + h) * kD + c_dim] = __float2half_rn(y);
           }
         }
       }
@@ -447,6 +450,70 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Combine the FP16 split partials (each O_s / l_s) of one query: for head h,
+// M = max(sink, m_s), w_s = l_s e^(m_s - M) / (e^(sink - M) + sum l_s
+// e^(m_s - M)), o = sum_s w_s (O_s / l_s) in split order, then the inverse
+// RoPE and a BF16 store.  grid (queries, n_heads / 8), 256 threads: warp =
+// head, lane = 16 dims.
+__global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__ ws_o, const float* __restrict__ ws_ml,
+                                                      int n_splits, int n_heads, const float* __restrict__ sink,
+                                                      const int32_t* __restrict__ q_pos0, int T, float theta,
+                                                      uint16_t* __restrict__ out) {
+  const int qi = blockIdx.x;
+  const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int bs = qi / T, tq = qi % T;
+  const int64_t t = (int64_t)q_pos0[bs] + tq;
+  const float sg = sink[h];
+  float M = sg;
+  for (int sp = 0; sp < n_splits; ++sp) M = fmaxf(M, ws_ml[(((int64_t)qi * n_splits + sp) * n_heads + h) * 2]);
+  float den = expf(sg - M);
+  for (int sp = 0; sp < n_splits; ++sp) {
+    const int64_t b2 = (((int64_t)qi * n_splits + sp) * n_heads + h) * 2;
+    const float ms = ws_ml[b2];
+    if (ms != -INFINITY) den += ws_ml[b2 + 1] * expf(ms - M);
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const int c0 = 16 * lane;
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  for (int sp = 0; sp < n_splits; ++sp) {
+    const int64_t b2 = (((int64_t)qi * n_splits + sp) * n_heads + h) * 2;
+    const float ms = ws_ml[b2];
+    if (ms == -INFINITY) continue;
+    const float a = ws_ml[b2 + 1] * expf(ms - M) * inv;
+    const uint4* src = reinterpret_cast<const uint4*>(ws_o + (((int64_t)qi * n_splits + sp) * n_heads + h) * kD + c0);
+    const uint4 v0 = src[0], v1 = src[1];
+    const __half2* h0 = reinterpret_cast<const __half2*>(&v0);
+    const __half2* h1 = reinterpret_cast<const __half2*>(&v1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f0 = __half22float2(h0[e]), f1 = __half22float2(h1[e]);
+      acc[2 * e] = fmaf(a, f0.x, acc[2 * e]);
+      acc[2 * e + 1] = fmaf(a, f0.y, acc[2 * e + 1]);
+      acc[8 + 2 * e] = fmaf(a, f1.x, acc[8 + 2 * e]);
+      acc[8 + 2 * e + 1] = fmaf(a, f1.y, acc[8 + 2 * e + 1]);
+    }
+  }
+  if (c0 >= kNope) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float cs, sn;
+      rope_cos_sin(-(double)t, (c0 - kNope) / 2 + e, kR, (double)theta, &cs, &sn);
+      const float x = acc[2 * e], y = acc[2 * e + 1];
+      acc[2 * e] = x * cs - y * sn;
+      acc[2 * e + 1] = x * sn + y * cs;
+    }
+  }
+  uint32_t o[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    o[e] = (uint32_t)f32_to_bf16_bits(acc[2 * e]) | ((uint32_t)f32_to_bf16_bits(acc[2 * e + 1]) << 16);
+  uint4* dst = reinterpret_cast<uint4*>(out + ((int64_t)qi * n_heads + h) * kD + c0);
+  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -499,8 +566,11 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
   const int rps = attn_tc_rows_per_split(total, T, dense);
   const int n_splits = (total + rps - 1) / rps;
   const int nhg = p.n_heads / kHg;
-  float* ws_o = ws;
-  float* ws_ml = ws ? ws + (size_t)nq * n_splits * p.n_heads * p.d : nullptr;
+  // workspace: FP16 partials O/l, then (max, sum) per (query, split, head)
+  const size_t n_part = (size_t)nq * n_splits * p.n_heads;
+  __half* ws_o = reinterpret_cast<__half*>(ws);
+  float* ws_ml = ws ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((n_part * p.d * 2 + 15) & ~(size_t)15))
+                    : nullptr;
   const size_t smem = attn_tc_smem_bytes();
   auto kfn = dense ? attn_tc<true> : attn_tc<false>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -512,7 +582,9 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
                                      sink, rps, n_splits, reinterpret_cast<uint16_t*>(out), ws_o, ws_ml, err);
   e = cudaGetLastError();
   if (e != cudaSuccess || n_splits == 1) return e;
-  return launch_attn_merge(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out, st);
+  attn_merge_f16<<<dim3(nq, p.n_heads / 8), 256, 0, st>>>(ws_o, ws_ml, n_splits, p.n_heads, sink, q_pos0, T,
+                                                          p.rope_theta, reinterpret_cast<uint16_t*>(out));
+  return cudaGetLastError();
 }
 
 size_t attn_tc_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense) {
@@ -520,7 +592,8 @@ size_t attn_tc_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense
   const int rps = attn_tc_rows_per_split(total, T, dense);
   const int n_splits = (total + rps - 1) / rps;
   if (n_splits == 1) return 0;
-  return (size_t)p.B * T * n_splits * p.n_heads * (p.d + 2) * sizeof(float);
+  const size_t n_part = (size_t)p.B * T * n_splits * p.n_heads;
+  return ((n_part * p.d * 2 + 15) & ~(size_t)15) + n_part * 2 * sizeof(float);
 }
 
 }  // namespace csa

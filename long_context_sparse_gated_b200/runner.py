@@ -95,10 +95,22 @@ class DeviceWorkload:
         hca_dense_attn(self.params, self.q, self.kv, self.kv_scale, self.win, self.win_scale, self.sink,
                        self.q_pos0, self.T, self.n_max, self.out, self.ws_attn, self.err, stream)
 
-    def csa_step(self, stream=None):
-        self.compress(stream)
-        self.index_topk(stream)
-        self.sparse_attn(stream)
+    def csa_step(self, stream=None, side=None):
+        """compress -> index + top-k -> sparse attention.  With a `side`
+        stream the compressor runs concurrently with the indexer (they are
+        independent; only the attention reads the new entry)."""
+        if side is None or not self.S:
+            self.compress(stream)
+            self.index_topk(stream)
+            self.sparse_attn(stream)
+            return
+        main = stream if stream is not None else torch.cuda.current_stream()
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            self.compress(side)
+        self.index_topk(main)
+        main.wait_stream(side)
+        self.sparse_attn(main)
 
     def hca_step(self, stream=None):
         self.compress(stream)
