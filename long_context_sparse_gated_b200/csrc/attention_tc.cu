@@ -144,8 +144,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   const int j = quad * 32 + lane;            // tile row of this thread
   const int qi = blockIdx.x, split = blockIdx.y, hg = blockIdx.z;
   const int bs = qi / T, tq = qi % T;
-  const int64_t t = (int64_t)q_pos0[bs] + tq;
-  const int64_t n_t = (t + 1) / m;
   const int h0 = hg * kHg;
   const int total = n_sel + W;
   const int sb = split * rows_per_split;
@@ -172,6 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  const int64_t t = (int64_t)q_pos0[bs] + tq;
+  const int64_t n_t = (t + 1) / m;
   const uint32_t tmem = S.tmem_base;
   const uint32_t s_col = tmem;         // S^T: 64 columns
   const uint32_t o_col = tmem + 64;    // O^T block b: columns 64 + 64 b
@@ -387,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     }
   }
 
+  pdl_trigger();
   // -- epilogue
   if (n_tiles > 0) sm100::mbar_wait(&S.bar_o, (n_tiles - 1) & 1, abort);
   sm100::tc_fence_after();
@@ -461,6 +463,7 @@ __global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__
                                                       int n_splits, int n_heads, const float* __restrict__ sink,
                                                       const int32_t* __restrict__ q_pos0, int T, float theta,
                                                       uint16_t* __restrict__ out) {
+  pdl_wait();
   const int qi = blockIdx.x;
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int bs = qi / T, tq = qi % T;
@@ -576,15 +579,14 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(nq, n_splits, nhg);
-  kfn<<<grid, kThreads, smem, st>>>(tq, reinterpret_cast<const uint8_t*>(cache.rows), cache.scale, cache.cap,
-                                     reinterpret_cast<const uint8_t*>(win.rows), win.scale, win.cap, idx, p.topk,
-                                     q_pos0, T, p.m, p.window, n_sel, p.n_heads, p.softmax_scale, p.rope_theta,
-                                     sink, rps, n_splits, reinterpret_cast<uint16_t*>(out), ws_o, ws_ml, err);
-  e = cudaGetLastError();
+  e = launch_pdl(kfn, grid, dim3(kThreads), smem, st, tq, reinterpret_cast<const uint8_t*>(cache.rows), cache.scale,
+                 cache.cap, reinterpret_cast<const uint8_t*>(win.rows), win.scale, win.cap, idx, p.topk, q_pos0, T,
+                 p.m, p.window, n_sel, p.n_heads, p.softmax_scale, p.rope_theta, sink, rps, n_splits,
+                 reinterpret_cast<uint16_t*>(out), ws_o, ws_ml, err);
   if (e != cudaSuccess || n_splits == 1) return e;
-  attn_merge_f16<<<dim3(nq, p.n_heads / 8), 256, 0, st>>>(ws_o, ws_ml, n_splits, p.n_heads, sink, q_pos0, T,
-                                                          p.rope_theta, reinterpret_cast<uint16_t*>(out));
-  return cudaGetLastError();
+  return launch_pdl(attn_merge_f16, dim3(nq, p.n_heads / 8), dim3(256), 0, st, (const __half*)ws_o,
+                    (const float*)ws_ml, n_splits, p.n_heads, sink, q_pos0, T, p.rope_theta,
+                    reinterpret_cast<uint16_t*>(out));
 }
 
 size_t attn_tc_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense) {

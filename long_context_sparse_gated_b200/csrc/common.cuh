@@ -47,6 +47,14 @@ __device__ __forceinline__ float ue8m0_to_f32(uint32_t e) {
   return __uint_as_float(e << 23);
 }
 
+// Programmatic dependent launch.  Kernels launched with launch_pdl() may
+// start while the previous kernel on the stream is finishing; pdl_wait()
+// blocks until that kernel has completed and its memory is visible, so every
+// kernel calls it before reading any global input.  pdl_trigger() lets the
+// next kernel's CTAs be scheduled early (they still wait in pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void raise_err(int32_t* err, int32_t bits) {
   if (err) atomicOr(err, bits);
 }

@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(1024) compress_kernel(
   float* part = smem + 2 * m;         // [G][d] partial sums
   __shared__ float red[32];
 
+  pdl_wait();
+  pdl_trigger();
   const int bs = blockIdx.y;
   const int64_t e = (int64_t)e_begin[bs] + blockIdx.x;
   if (e >= e_end[bs]) return;
@@ -166,14 +168,11 @@ cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, c
   dim3 grid(max_entries, p.B);
   const bool f32 = p.act_fmt == CSA_ACT_F32, kv32 = p.kv_fmt == CSA_KV_F32;
   auto* rows = reinterpret_cast<uint8_t*>(out.rows);
-  if (f32 && kv32)
-    compress_kernel<true, true><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
-  else if (f32)
-    compress_kernel<true, false><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
-  else if (kv32)
-    compress_kernel<false, true><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
-  else
-    compress_kernel<false, false><<<grid, threads, smem, st>>>(p, a, b, gate, S, tok_base, e_begin, e_end, norm_w, rows, out.scale, out.cap, out_pos, err);
+  auto kfn = f32 ? (kv32 ? compress_kernel<true, true> : compress_kernel<true, false>)
+                 : (kv32 ? compress_kernel<false, true> : compress_kernel<false, false>);
+  cudaError_t e = launch_pdl(kfn, grid, dim3(threads), smem, st, p, a, b, gate, S, tok_base, e_begin, e_end, norm_w,
+                             rows, out.scale, out.cap, out_pos, err);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = S.tmem_base;
+  pdl_wait();  // inputs may come from the previous kernel on the stream
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -294,6 +295,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     }
   }
 
+  pdl_trigger();
   sm100::tc_fence_before();
   __syncthreads();
   if (S.abort && threadIdx.x == 0) raise_err(err, CSA_DEV_ERR_TIMEOUT);
@@ -388,8 +390,9 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(index_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  index_scores_tc<<<grid, kThreadsTc, smem, st>>>(tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap, nq, n_max, scores, ld,
-                                           hist, err);
+  e = launch_pdl(index_scores_tc, dim3(grid), dim3(kThreadsTc), smem, st, tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap,
+                 nq, n_max, scores, ld, hist, err);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -9,6 +9,25 @@
 
 namespace csa {
 
+// Launch with programmatic stream serialisation (see pdl_wait in
+// common.cuh): the kernel may begin while its predecessor on the stream
+// drains.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, const float* gate,
                             int64_t S, const int32_t* tok_base, const int32_t* e_begin,
                             const int32_t* e_end, int32_t max_entries, const float* norm_w,

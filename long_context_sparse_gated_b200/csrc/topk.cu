@@ -257,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_select(const float* __restri
                                                             const int* __restrict__ ccount, int n_chunks) {
   extern __shared__ uint8_t smem_raw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
   const int qi = blockIdx.x;
   const int bs = qi / T, tq = qi % T;
   const int64_t t = (int64_t)q_pos0[bs] + tq;
@@ -362,6 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_collect(const float* __restr
                                                              int n_chunks) {
   extern __shared__ uint8_t smem_raw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
   const int qi = blockIdx.x, chunk = blockIdx.y;
   const int bs = qi / T, tq = qi % T;
   const int64_t t = (int64_t)q_pos0[bs] + tq;
@@ -423,16 +427,15 @@ cudaError_t launch_topk_select(const csa_params& p, const float* scores, int ld,
     ccount = reinterpret_cast<int*>(ckey + (size_t)nq * chunks * kCap);
     cudaError_t e = cudaFuncSetAttribute(topk_collect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_collect<<<dim3(nq, chunks), kThreads, smem, st>>>(scores, ld, n_max, hist, q_pos0, T, p.m, p.topk, cidx,
-                                                           ckey, ccount, chunks);
-    e = cudaGetLastError();
+    e = launch_pdl(topk_collect, dim3(nq, chunks), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T,
+                   p.m, p.topk, cidx, ckey, ccount, chunks);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e = cudaFuncSetAttribute(topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_select<<<nq, kThreads, smem, st>>>(scores, ld, n_max, hist, q_pos0, T, p.m, p.topk, out_idx, cidx, ckey,
-                                          ccount, ccount ? chunks : 0);
-  return cudaGetLastError();
+  return launch_pdl(topk_select, dim3(nq), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T, p.m,
+                    p.topk, out_idx, (const int*)cidx, (const uint32_t*)ckey, (const int*)ccount,
+                    ccount ? chunks : 0);
 }
 
 }  // namespace csa
