@@ -109,6 +109,24 @@ struct VisibleCache {
 
 constexpr int kThreadsTc = 64 + 128 * kEpiGroups;  // producer, MMA, 2 epilogue warpgroups
 
+// Walks the CTA's tile range as (query, block) pairs.  One 64-bit division
+// at the start; afterwards a step is an increment, so the single-thread
+// producer and MMA loops do not pay a division latency per tile.
+struct TileCursor {
+  int64_t t, end;
+  int qi, j, tpq;
+  __device__ __forceinline__ TileCursor(int64_t begin, int64_t e, int tiles_per_query)
+      : t(begin), end(e), tpq(tiles_per_query) {
+    qi = (int)(begin / tiles_per_query);
+    j = (int)(begin - (int64_t)qi * tiles_per_query);
+  }
+  __device__ __forceinline__ bool more() const { return t < end; }
+  __device__ __forceinline__ void next() {
+    ++t;
+    if (++j == tpq) { j = 0; ++qi; }
+  }
+};
+
 __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     const __grid_constant__ CUtensorMap tm_key, const __grid_constant__ CUtensorMap tm_q,
     const __grid_constant__ CUtensorMap tm_sfk, const __grid_constant__ CUtensorMap tm_sfq,
@@ -160,10 +178,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       uint32_t it = 0, nq = 0;
       int cur_q = -1;
       VisibleCache vc;
-      for (int64_t t = t_begin; t < t_end; ++t) {
-        const int qi = (int)(t / tpq), j = (int)(t % tpq);
+      int bs = 0;
+      for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
+        const int qi = c.qi, j = c.j;
         if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
         if (qi != cur_q) {  // the query's 64 heads, once per query
+          bs = qi / T;
           const int sl = nq & 1;
           if (!sm100::mbar_wait(&S.qempty[sl], ((nq >> 1) & 1) ^ 1, abort)) break;
           sm100::mbar_arrive_expect_tx(&S.qfull[sl], kQueryTx);
@@ -177,7 +197,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         if (!sm100::mbar_wait(&S.empty[s], ph ^ 1, abort)) break;
         Stage& st = S.st[s];
         sm100::mbar_arrive_expect_tx(&S.full[s], kStageTx);
-        const int64_t row = (int64_t)(qi / T) * k_cap + (int64_t)j * kTileM;
+        const int64_t row = (int64_t)bs * k_cap + (int64_t)j * kTileM;
         sm100::tma_load_3d(st.key, &tm_key, &S.full[s], 0, (int32_t)(row / 4), 0);
         sm100::tma_load_1d(st.sfk, &tm_sfk, &S.full[s], (int32_t)row);
         ++it;
@@ -188,8 +208,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     uint32_t it = 0, nq = 0;
     int cur_q = -1, sl = 0;
     VisibleCache vc;
-    for (int64_t t = t_begin; t < t_end; ++t) {
-      const int qi = (int)(t / tpq), j = (int)(t % tpq);
+    for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
+      const int qi = c.qi, j = c.j;
       if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
       if (qi != cur_q) {
         // the previous query's slot is free once its MMAs complete
@@ -255,8 +275,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     int wq = -1;
     float wv[kHeads];
     VisibleCache vc;
-    for (int64_t t = t_begin; t < t_end; ++t) {
-      const int qi = (int)(t / tpq), j = (int)(t % tpq);
+    for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
+      const int qi = c.qi, j = c.j;
       const int n_t = vc.get(q_pos0, T, m, qi, n_max);
       if (j * kTileM >= n_t) continue;
       const uint32_t my = it++;
