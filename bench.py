@@ -97,6 +97,30 @@ def launches_per_step(w):
     return n
 
 
+def graph_kernel_nodes(graph):
+    """Kernel nodes of a captured CUDA graph (driver API on the raw handle);
+    None when the handle or the driver call is not available."""
+    try:
+        import ctypes
+        drv = ctypes.CDLL("libcuda.so.1")
+        h = ctypes.c_void_p(graph.raw_cuda_graph())
+        n = ctypes.c_size_t(0)
+        if drv.cuGraphGetNodes(h, None, ctypes.byref(n)) != 0:
+            return None
+        nodes = (ctypes.c_void_p * n.value)()
+        if drv.cuGraphGetNodes(h, nodes, ctypes.byref(n)) != 0:
+            return None
+        kernels = 0
+        for i in range(n.value):
+            t = ctypes.c_int(-1)
+            if drv.cuGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t)) != 0:
+                return None
+            kernels += t.value == 0  # CU_GRAPH_NODE_TYPE_KERNEL
+        return kernels
+    except Exception:
+        return None
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
 
@@ -289,6 +313,7 @@ def main():
     # dominant call, the rest) so that host launch cost does not starve the
     # device; events between the replays time the dominant call alone.
     graphs = []
+    kernels_per_step = None  # counted from the captured graphs when possible
     if not args.no_graph:
         cap = torch.cuda.Stream()
         cap.wait_stream(stream)
@@ -299,13 +324,19 @@ def main():
                 for fn in phases:
                     g = None
                     if fn is not None:
-                        g = torch.cuda.CUDAGraph()
+                        try:
+                            g = torch.cuda.CUDAGraph(keep_graph=True)
+                        except TypeError:
+                            g = torch.cuda.CUDAGraph()
                         with torch.cuda.graph(g, stream=cap):
                             fn(cap)
                     parts.append(g)
             graphs.append(parts)
         stream.wait_stream(cap)
         torch.cuda.synchronize()
+        counts = [graph_kernel_nodes(g) for g in graphs[0] if g is not None]
+        if counts and all(c is not None for c in counts):
+            kernels_per_step = sum(counts)
 
     def timed_step(i, ev=None):
         if not graphs:
@@ -412,7 +443,8 @@ def main():
         "config": {"workload": CONFIG_NAMES[args.config], "name": args.config, "batch": p.B,
                    "context": int(w["L"].max()), "queries_per_step": queries,
                    "l2": f"inputs larger than L2: {n_copies} device copies rotated, {n_copies * step_bytes / 2**20:.0f} MiB per cycle"},
-        "gpu_launches": args.steps * launches_per_step(w),
+        "gpu_launches": args.steps * (kernels_per_step if kernels_per_step is not None else launches_per_step(w)),
+        "gpu_launches_source": "graph kernel nodes" if kernels_per_step is not None else "static count",
         "graphs": not args.no_graph,
         "roofline": {"bound": "hbm", "kernel": "csa_index_topk" if p.k > 0 else "hca_dense_attn",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,

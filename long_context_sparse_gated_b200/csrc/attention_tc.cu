@@ -8,26 +8,34 @@
 // One CTA = one query, one group of 64 heads, one split of its candidate
 // slots (entries, then window tokens), in 128-row tiles:
 //
-//   gather    8 warps load the tile's 128 rows (16-byte loads of the
-//             576-byte FP8/BF16 rows), convert them to FP16 and store them
-//             as a 128-row x 512-dim K-major tile (128-byte swizzle).  E4M3
-//             codes are exact in FP16; the RoPE dims are stored divided by
-//             the row scale s_j, so that  s_j * (V'_j . q) = v_j . q  and one
-//             accumulator holds a whole logit.  FP16 (10-bit mantissa) keeps
-//             the rounding of P' and of the scaled RoPE dims 8x below BF16's.
+//   resolve   128 threads map the tile's slots to cache / window rows
+//   gather    the same threads each issue one 576-byte bulk copy (TMA
+//             engine, no tensor map) of their row into a staging area and
+//             load the row's scale; while the copies are in flight the
+//             BF16 query (TMA) is converted to FP16 in place; then the
+//             rows are read from the staging area, converted to FP16 and
+//             stored as a
+//             128-row x 512-dim K-major tile (128-byte swizzle).  E4M3 codes
+//             are exact in FP16; the RoPE dims are stored divided by the row
+//             scale s_j, so that  s_j * (V'_j . q) = v_j . q  and one
+//             accumulator holds a whole logit.
 //   S^T       tcgen05.mma kind::f16 (FP16 A/B, FP32 accumulate):
 //             S^T[j, h] = sum_c V'[j, c] Q[h, c]
-//             (M = 128 rows, N = 64 heads, K = 512) into TMEM
+//             (M = 128 rows, N = 64 heads, K = 512) into TMEM, 32
+//             back-to-back MMAs from precomputed descriptors
 //   softmax   per row thread: z = tau * s_j * S^T; per-head tile maxima and
 //             sums by warp-transposed shuffles; the running max is raised
 //             lazily (only when a tile exceeds it by > 8), so O is rarely
-//             rescaled; P'^T[h, j] = exp(z - m_h) * s_j in FP16 to smem
-//   O^T       tcgen05.mma: O^T[c, h] += sum_j V'[j, c] P'[h, j]
-//             (A = V'^T, the same tile read MN-major; M = 128 dims x 4
-//             blocks, N = 64 heads, K = 128 rows) into TMEM
-//   epilogue  normalise with the sink term, inverse RoPE, BF16 store -- or,
-//             with several splits, write the partial O/l (FP16) and (m, l)
-//             that attn_merge_f16 combines in split order.
+//             rescaled; P' = exp(z - m_h) * s_j in FP16, stored MN-major
+//             (each row thread writes its 32 heads as four 16-byte words)
+//   O^T       tcgen05.mma: O^T[c, h] += sum_j V'[j, c] P'[j, h]
+//             (A = V'^T, the same tile read MN-major; B = P' MN-major;
+//             M = 128 dims x 4 blocks, N = 64 heads, K = 128 rows)
+//   epilogue  normalise (with the sink term when the split is the whole
+//             row set), inverse RoPE, then the 64 x 512 result is staged in
+//             shared memory and written with coalesced 16-byte stores: the
+//             BF16 output, or with several splits the FP16 partial O/l and
+//             (m, l) that attn_merge_f16 combines in split order.
 //
 // 8 warps (two per TMEM lane quadrant) gather, run the softmax and the
 // epilogue; thread 0 also issues the query TMA and the MMAs between block
@@ -50,28 +58,47 @@ constexpr int kNope = kD - kR;             // 448
 constexpr int kRowBytes = kNope + 2 * kR;  // 576
 constexpr int kChunks = kRowBytes / 16;    // 36 16-byte chunks per stored row
 constexpr int kThreads = 256;             // 8 warps: two per TMEM lane quadrant
-constexpr float kLazy = 8.0f;  // raise the running max only past +8 (e^8 < 3000)
+constexpr int kLoads = kRows * kChunks / kThreads;  // 18 loads per thread per tile
+static_assert(kRows * kChunks % kThreads == 0, "gather must divide evenly");
+static_assert(kChunks == 36 && (kRows / 8) * (kChunks / 4) == 8 * kLoads, "conversion pairs cover the tile");
+constexpr float kLog2e = 1.4426950408889634f;
+// logits are kept in base-2 units (z * log2 e) so that probabilities are
+// exp2f of a difference; the running max is raised only when a tile exceeds
+// it by more than 11.5 (2^11.5 < 3000), so O is rarely rescaled
+constexpr float kLazy = 11.5f;
 constexpr uint32_t kTmemCols = 512;        // S^T: 64, O^T: 4 x 64
 
 struct __align__(1024) AttnSmem {
-  uint8_t v[8][kRows * 128];  // 8 K-chunks of 64 dims: [128 rows][128 B], 128B swizzle
+  uint8_t v[8][kRows * 128];  // 8 K-chunks of 64 dims: [128 rows][128 B], 128B swizzle;
+                              // after the last tile: the [64 heads][512 dims] output stage
+  uint8_t p[kRows * 128];     // P' MN-major: [128 rows][64 heads] FP16, 128B swizzle
   uint8_t q[8][kHg * 128];    // 8 K-chunks: [64 heads][128 B]
-  uint8_t p[2][kHg * 128];    // P'^T: 2 K-chunks of 64 rows: [64 heads][128 B]
   float scale[kRows];
   float inv_scale[kRows];
-  int64_t rowoff[kRows];      // byte offset of the row, -1 when the slot is empty
-  int src[kRows];             // 1 cache, 2 window
+  int live[kRows];            // row takes part (non-empty slot with a valid scale)
   float red[8][64];
   float mh[kHg], lh[kHg], alpha[kHg];
-  uint64_t bar_q, bar_s, bar_o;
+  float rope_c[kR / 2], rope_s[kR / 2];  // inverse-RoPE rotation of this query
+  uint64_t bar_q, bar_g, bar_s, bar_o;
   uint32_t tmem_base;
   int abort;
   int rescale;
 };
 
+// The raw rows of a tile (128 x 576 B) are staged in V' chunks 4..7 and the
+// P' buffer that follows them; both are free while a tile is gathered.
+constexpr int kStageOff = 4 * kRows * 128;
+static_assert(offsetof(AttnSmem, p) == sizeof(((AttnSmem*)0)->v), "P' must follow V'");
+static_assert(kStageOff + kRows * kRowBytes <= (int)(sizeof(((AttnSmem*)0)->v) + sizeof(((AttnSmem*)0)->p)),
+              "staging area");
+
 __device__ __forceinline__ uint32_t sw128(int row, int chunk16) {
   return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
+
+// descriptor + byte offset (start-address field, 16-byte units; shared
+// addresses stay below 2^18, so the 14-bit field does not overflow)
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
 
 // 16 E4M3 codes -> 16 FP16 (exact), as two 16-byte words
 __device__ __forceinline__ void e4m3x16_to_f16(const uint4& in, uint4& lo, uint4& hi) {
@@ -108,6 +135,11 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4& in) {
   return bf16x8_scale_to_f16(in, 1.0f);
 }
 
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  const __half2 r = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // max / sum over the 32 lanes of a warp for each of 32 values: afterwards
 // lane l holds the reduction of value index l.
 template <bool kMax>
@@ -125,6 +157,32 @@ __device__ __forceinline__ float warp_transpose_reduce32(float (&v)[32]) {
     }
   }
   return v[0];
+}
+
+// Row of candidate slot `slot` (< se) of query t: src 1 = cache row, 2 =
+// window ring row, 0 = empty; *off = element row index into that array.
+template <bool kDense>
+__device__ __forceinline__ int resolve_slot(int slot, int se, int n_sel, int64_t t, int64_t n_t, int W, int bs, int qi,
+                                            const int32_t* __restrict__ idx, int topk, int64_t cache_cap,
+                                            int64_t win_cap, int32_t* err, int64_t* off) {
+  int src = 0;
+  int64_t row = 0;
+  if (slot < se) {
+    if (slot < n_sel) {
+      if (kDense) {
+        if (slot < n_t && slot < cache_cap) { src = 1; row = slot; }
+      } else {
+        const int e = idx[(int64_t)qi * topk + slot];
+        if (e >= 0 && e < n_t && e < cache_cap) { src = 1; row = e; }
+        else if (e != -1) raise_err(err, CSA_DEV_ERR_INDEX);
+      }
+    } else {
+      const int64_t pos = t - W + 1 + (slot - n_sel);
+      if (pos >= 0) { src = 2; row = pos % win_cap; }
+    }
+  }
+  *off = src == 1 ? (int64_t)bs * cache_cap + row : (src == 2 ? (int64_t)bs * win_cap + row : -1);
+  return src;
 }
 
 template <bool kDense>
@@ -149,11 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   const int sb = split * rows_per_split;
   const int se = min(total, sb + rows_per_split);
   const int n_tiles = (se - sb + kRows - 1) / kRows;
+  const bool single = n_splits == 1;
   volatile int* abort = &S.abort;
   const bool issuer = threadIdx.x == 0;
 
   if (issuer) {
     sm100::mbar_init(&S.bar_q, 1);
+    sm100::mbar_init(&S.bar_g, 1);
     sm100::mbar_init(&S.bar_s, 1);
     sm100::mbar_init(&S.bar_o, 1);
     S.abort = 0;
@@ -181,8 +241,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     sm100::mbar_arrive_expect_tx(&S.bar_q, 8 * kHg * 128);
     for (int c = 0; c < 8; ++c) sm100::tma_load_2d(S.q[c], &tm_q, &S.bar_q, 64 * c, qi * n_heads + h0);
   }
+  // the inverse-RoPE rotation by -t of the 32 RoPE pairs, once per CTA
+  if (single && wt >= 64 && wt < 64 + kR / 2) {
+    float c, sn;
+    rope_cos_sin(-(double)t, wt - 64, kR, (double)theta, &c, &sn);
+    S.rope_c[wt - 64] = c;
+    S.rope_s[wt - 64] = sn;
+  }
   const uint32_t idS = sm100::idesc_f16(kRows, kHg, 0, 0);
-  const uint32_t idO = sm100::idesc_f16(128, kHg, 1, 0);
+  const uint32_t idO = sm100::idesc_f16(128, kHg, 1, 1);
+  // K-major V' (A of S^T), K-major Q (B of S^T), MN-major V'^T (A of O^T:
+  // 64-dim atoms 16 KB apart, 8-row groups 1 KB apart), MN-major P' (B of
+  // O^T: one 64-head atom, 8-row groups 1 KB apart)
+  const uint64_t dV = sm100::smem_desc(sm100::smem_u32(S.v[0]), 16, 1024, 2);
+  const uint64_t dQ = sm100::smem_desc(sm100::smem_u32(S.q[0]), 16, 1024, 2);
+  const uint64_t dVt = sm100::smem_desc(sm100::smem_u32(S.v[0]), kRows * 128, 1024, 2);
+  const uint64_t dP = sm100::smem_desc(sm100::smem_u32(S.p), kRows * 128, 1024, 2);
+
+  // Row of this thread (wt < kRows) in the current tile, resolved one tile
+  // ahead: while tile i is computed, tile i+1's rows are resolved, their
+  // scales loaded and their bytes prefetched into L2.
+  int my_src = 0;
+  int64_t my_off = -1;
+  float my_sc = 1.f;
+  if (wt < kRows && n_tiles > 0) {
+    my_src = resolve_slot<kDense>(sb + wt, se, n_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap, err, &my_off);
+    if (my_src == 1) my_sc = cache_scale[my_off];
+    if (my_src == 2) my_sc = win_scale[my_off];
+  }
 
   // Control flow is uniform across the CTA (every __syncthreads is reached
   // by all threads); a failed bounded wait only raises the abort flag,
@@ -191,94 +277,93 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     const int tb = sb + i * kRows;
     if (i > 0) sm100::mbar_wait(&S.bar_o, (i - 1) & 1, abort);  // V' and P' buffers free
     if (wt == 0) S.rescale = 0;
-    // -- resolve the tile's rows
+    const int n_copy = __syncthreads_count(my_src != 0);
+    if (issuer) sm100::mbar_arrive_expect_tx(&S.bar_g, (uint32_t)(n_copy * kRowBytes));
+    __syncthreads();
+    // -- gather: one bulk copy per non-empty row (rows and the staging area
+    //    are 16-byte aligned, 576 = 36 x 16 bytes)
+    uint8_t* stg = &S.v[0][0] + kStageOff;
+    if (my_src) {
+      const uint8_t* src = (my_src == 2 ? win_rows : cache_rows) + my_off * kRowBytes;
+      sm100::bulk_load(stg + wt * kRowBytes, src, kRowBytes, &S.bar_g);
+    }
     if (wt < kRows) {
-      const int slot = tb + wt;
-      int src = 0;
-      int64_t row = 0;
-      if (slot < se) {
-        if (slot < n_sel) {
-          if (kDense) {
-            if (slot < n_t && slot < cache_cap) { src = 1; row = slot; }
-          } else {
-            const int e = idx[(int64_t)qi * topk + slot];
-            if (e >= 0 && e < n_t && e < cache_cap) { src = 1; row = e; }
-            else if (e != -1) raise_err(err, CSA_DEV_ERR_INDEX);
-          }
-        } else {
-          const int64_t pos = t - W + 1 + (slot - n_sel);
-          if (pos >= 0) { src = 2; row = pos % win_cap; }
-        }
-      }
-      float sc = 1.f;
-      int64_t off = -1;
-      if (src == 1) { off = ((int64_t)bs * cache_cap + row); sc = cache_scale[off]; }
-      if (src == 2) { off = ((int64_t)bs * win_cap + row); sc = win_scale[off]; }
+      float sc = my_sc;
+      int live = my_src != 0;
       if (!(sc > 0.f) || !(sc < INFINITY)) {  // scales are positive and finite by construction
-        if (src) raise_err(err, CSA_DEV_ERR_RANGE);
-        src = 0;
-        off = -1;
+        if (my_src) raise_err(err, CSA_DEV_ERR_RANGE);
+        live = 0;  // the row is dropped (zeroed below)
         sc = 1.f;
       }
-      S.src[wt] = src;
-      S.rowoff[wt] = off < 0 ? -1 : off * kRowBytes;
+      S.live[wt] = live;
       S.scale[wt] = sc;
       S.inv_scale[wt] = 1.f / sc;
-    }
-    __syncthreads();
-    // -- gather + convert: 128 rows x 36 chunks of 16 B, 18 per thread in
-    //    two batches of 9 loads in flight
-#pragma unroll
-    for (int bt = 0; bt < 2; ++bt) {
-      uint4 raw[9];
-#pragma unroll
-      for (int k = 0; k < 9; ++k) {
-        const int u = wt + kThreads * (9 * bt + k);
-        const int r = u / kChunks, c = u % kChunks;
-        const int64_t off = S.rowoff[r];
-        const uint8_t* base = S.src[r] == 2 ? win_rows : cache_rows;
-        raw[k] = off >= 0 ? __ldg(reinterpret_cast<const uint4*>(base + off) + c) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int k = 0; k < 9; ++k) {
-        const int u = wt + kThreads * (9 * bt + k);
-        const int r = u / kChunks, c = u % kChunks;
-        if (c < kNope / 16) {
-          // dims 16c .. 16c+15 -> K-chunk (16c)/64, 16-byte slots 2(c%4), 2(c%4)+1
-          uint4 lo, hi;
-          e4m3x16_to_f16(raw[k], lo, hi);
-          uint8_t* ch = S.v[c >> 2];
-          *reinterpret_cast<uint4*>(ch + sw128(r, 2 * (c & 3))) = lo;
-          *reinterpret_cast<uint4*>(ch + sw128(r, 2 * (c & 3) + 1)) = hi;
-        } else {
-          // RoPE dims 448 + 8(c-28) .. : chunk 7, slot (c-28)
-          const uint4 v = bf16x8_scale_to_f16(raw[k], S.inv_scale[r]);
-          *reinterpret_cast<uint4*>(S.v[7] + sw128(r, c - kNope / 16)) = v;
-        }
-      }
     }
     if (i == 0) {
       // queries: BF16 (TMA) -> FP16 in place, same swizzled positions
       sm100::mbar_wait(&S.bar_q, 0, abort);
       uint4* qv = reinterpret_cast<uint4*>(&S.q[0][0]);
+#pragma unroll 4
       for (int e = wt; e < 8 * kHg * 128 / 16; e += kThreads) qv[e] = bf16x8_to_f16(qv[e]);
+    }
+    // Conversion work: (8-row block, group of four 16-byte chunks) pairs,
+    // one pair per warp instruction, lane = 4 x row-in-block + chunk-in-group:
+    // both the staging reads and the swizzled V' stores then spread a warp's
+    // 32 x 16 bytes over all banks.
+    sm100::mbar_wait(&S.bar_g, i & 1, abort);
+    uint4 raw[kLoads];
+#pragma unroll
+    for (int k = 0; k < kLoads; ++k) {
+      const int pr = warp + 8 * k;
+      const int r = 8 * (pr / 9) + (lane >> 2), c = 4 * (pr % 9) + (lane & 3);
+      raw[k] = *reinterpret_cast<const uint4*>(stg + r * kRowBytes + c * 16);
+    }
+    __syncthreads();  // staging area read by all; scales and live flags visible
+    // -- convert + store V' (empty and dropped rows as zeros: the staging
+    //    area holds stale bytes there)
+#pragma unroll
+    for (int k = 0; k < kLoads; ++k) {
+      const int pr = warp + 8 * k;
+      const int r = 8 * (pr / 9) + (lane >> 2), c = 4 * (pr % 9) + (lane & 3);
+      const bool live = S.live[r] != 0;
+      if (c < kNope / 16) {
+        // dims 16c .. 16c+15 -> K-chunk (16c)/64, 16-byte slots 2(c%4), 2(c%4)+1
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+        if (live) e4m3x16_to_f16(raw[k], lo, hi);
+        uint8_t* ch = S.v[c >> 2];
+        *reinterpret_cast<uint4*>(ch + sw128(r, 2 * (c & 3))) = lo;
+        *reinterpret_cast<uint4*>(ch + sw128(r, 2 * (c & 3) + 1)) = hi;
+      } else {
+        // RoPE dims 448 + 8(c-28) .. : chunk 7, slot (c-28)
+        const uint4 v = live ? bf16x8_scale_to_f16(raw[k], S.inv_scale[r]) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(S.v[7] + sw128(r, c - kNope / 16)) = v;
+      }
     }
     sm100::fence_proxy_async_smem();
     __syncthreads();
     // -- S^T = V' Q^T over K = 512 (32 steps of 16)
     if (issuer) {
-      const bool ok = !*abort;
       sm100::tc_fence_after();
-      if (ok && !*abort) {
-#pragma unroll 1
+      if (!*abort) {
+#pragma unroll
         for (int kk = 0; kk < 32; ++kk) {
-          const int c = kk >> 2, o = (kk & 3) * 32;
-          const uint64_t a = sm100::smem_desc(sm100::smem_u32(S.v[c]) + o, 16, 1024, 2);
-          const uint64_t b = sm100::smem_desc(sm100::smem_u32(S.q[c]) + o, 16, 1024, 2);
-          sm100::mma_f16(s_col, a, b, idS, kk > 0);
+          const uint32_t o = (uint32_t)((kk >> 2) * kRows * 128 + (kk & 3) * 32);
+          const uint32_t oq = (uint32_t)((kk >> 2) * kHg * 128 + (kk & 3) * 32);
+          sm100::mma_f16(s_col, dadd(dV, o), dadd(dQ, oq), idS, kk > 0);
         }
         sm100::tc_commit(&S.bar_s);
       }
+    }
+    // -- next tile: resolve, scale load and L2 prefetch while this one runs
+    int nx_src = 0;
+    int64_t nx_off = -1;
+    float nx_sc = 1.f;
+    if (wt < kRows && i + 1 < n_tiles) {
+      nx_src = resolve_slot<kDense>(tb + kRows + wt, se, n_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap,
+                                    err, &nx_off);
+      if (nx_src) sm100::bulk_prefetch_l2((nx_src == 2 ? win_rows : cache_rows) + nx_off * kRowBytes, kRowBytes);
+      if (nx_src == 1) nx_sc = cache_scale[nx_off];
+      if (nx_src == 2) nx_sc = win_scale[nx_off];
     }
     sm100::mbar_wait(&S.bar_s, i & 1, abort);
     sm100::tc_fence_after();
@@ -290,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       sm100::tmem_ld_x16(ta, a);
       sm100::tmem_ld_x16(ta + 16, b);
       sm100::tmem_ld_wait();
-      const bool valid = S.src[j] != 0;
-      const float f = tau * S.scale[j];
+      const bool valid = S.live[j] != 0;
+      const float f = tau * kLog2e * S.scale[j];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         z[c] = valid ? f * __uint_as_float(a[c]) : -INFINITY;
@@ -316,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       if (i == 0) {
         S.mh[h] = tmax;
       } else if (tmax > mo + kLazy) {
-        al = (mo == -INFINITY) ? 0.f : expf(mo - tmax);
+        al = (mo == -INFINITY) ? 0.f : exp2f(mo - tmax);
         S.mh[h] = tmax;
         S.lh[h] *= al;
         resc = 1;
@@ -344,20 +429,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       }
       sm100::tmem_st_wait();
     }
-    // probabilities, P'^T stores and per-head sums
+    // probabilities, P' stores (row j, heads 32*half .. +31 = four 16-byte
+    // words) and per-head sums
     {
       const float sj = S.scale[j];
       float v[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const int h = 32 * half + c;
-        const float mh = S.mh[h];
-        const float pr = (mh == -INFINITY || z[c] == -INFINITY) ? 0.f : expf(z[c] - mh);
-        v[c] = pr;
-        // P'^T[h][j]: K-major, K-chunk j/64, row h, 16-byte slot ((j%64)/8)
-        const __half pb = __float2half_rn(pr * sj);
-        uint8_t* dst = S.p[j >> 6] + sw128(h, (j & 63) >> 3) + 2 * (j & 7);
-        *reinterpret_cast<__half*>(dst) = pb;
+        const float mh = S.mh[32 * half + c];
+        v[c] = (mh == -INFINITY || z[c] == -INFINITY) ? 0.f : exp2f(z[c] - mh);
+      }
+#pragma unroll
+      for (int w4 = 0; w4 < 4; ++w4) {
+        const int b = 8 * w4;
+        const uint4 pk = make_uint4(pack_half2(v[b] * sj, v[b + 1] * sj), pack_half2(v[b + 2] * sj, v[b + 3] * sj),
+                                    pack_half2(v[b + 4] * sj, v[b + 5] * sj), pack_half2(v[b + 6] * sj, v[b + 7] * sj));
+        *reinterpret_cast<uint4*>(S.p + sw128(j, 4 * half + w4)) = pk;
       }
       S.red[warp][lane] = warp_transpose_reduce32<false>(v);
     }
@@ -370,77 +457,101 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       for (int q4 = 0; q4 < 4; ++q4) ts += S.red[hh * 4 + q4][hl];
       S.lh[h] += ts;
     }
-    // -- O^T[blk] += V'^T[blk] P'^T over K = 128 rows (8 steps of 16)
+    // -- O^T[blk] += V'^T[blk] P' over K = 128 rows (8 steps of 16)
     if (issuer) {
       sm100::tc_fence_after();
       if (!*abort) {
-#pragma unroll 1
+#pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = sm100::smem_desc(sm100::smem_u32(S.v[2 * blk]) + kk * 2048, 16384, 1024, 2);
-            const uint64_t b = sm100::smem_desc(sm100::smem_u32(S.p[kk >> 2]) + (kk & 3) * 32, 16, 1024, 2);
-            sm100::mma_f16(o_col + 64 * blk, a, b, idO, (i > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t oa = (uint32_t)(2 * blk * kRows * 128 + kk * 2048);
+            sm100::mma_f16(o_col + 64 * blk, dadd(dVt, oa), dadd(dP, (uint32_t)(kk * 2048)), idO,
+                           (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
         sm100::tc_commit(&S.bar_o);
       }
     }
+    my_src = nx_src;
+    my_off = nx_off;
+    my_sc = nx_sc;
   }
 
   pdl_trigger();
   // -- epilogue
   if (n_tiles > 0) sm100::mbar_wait(&S.bar_o, (n_tiles - 1) & 1, abort);
   sm100::tc_fence_after();
-  __syncthreads();  // lh final; abort flag now uniform
+  __syncthreads();  // lh final; abort flag now uniform; V' free
+  // per-head output factor: single split, normalised with the sink term
+  // here; several splits, the partial normalised by its own sum (FP16) plus
+  // (max, sum)
+  if (wt < kHg) {
+    const float mh = S.mh[wt], lh = S.lh[wt];
+    float fh;
+    if (single) {
+      const float sg = sink[h0 + wt] * kLog2e;
+      const float ms = fmaxf(sg, mh);
+      const float den = exp2f(sg - ms) + (mh == -INFINITY ? 0.f : lh * exp2f(mh - ms));
+      fh = (mh == -INFINITY || !(den > 0.f)) ? 0.f : exp2f(mh - ms) / den;
+    } else {
+      fh = lh > 0.f ? 1.f / lh : 0.f;
+    }
+    S.alpha[wt] = fh;
+  }
+  __syncthreads();
   const bool ok = !S.abort;
-  const bool single = n_splits == 1;
   if (ok && n_tiles > 0) {
-    // single split: normalise with the sink term here; several splits: the
-    // partial normalised by its own sum, as FP16, plus (max, sum)
     float f[32];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const int h = 32 * half + c;
-      const float mh = S.mh[h], lh = S.lh[h];
-      if (single) {
-        const float sg = sink[h0 + h];
-        const float ms = fmaxf(sg, mh);
-        const float den = expf(sg - ms) + (mh == -INFINITY ? 0.f : lh * expf(mh - ms));
-        f[c] = (mh == -INFINITY || !(den > 0.f)) ? 0.f : expf(mh - ms) / den;
-      } else {
-        f[c] = lh > 0.f ? 1.f / lh : 0.f;
-      }
-    }
+    for (int c = 0; c < 32; ++c) f[c] = S.alpha[32 * half + c];
+    uint16_t* stage = reinterpret_cast<uint16_t*>(&S.v[0][0]);  // [64 heads][512 dims]
 #pragma unroll 1
-    for (int blk = 0; blk < 4; ++blk) {
-      const int c_dim = 128 * blk + quad * 32 + lane;
-      float cs = 1.f, sn = 0.f;
-      if (single && c_dim >= kNope) rope_cos_sin(-(double)t, (c_dim - kNope) >> 1, kR, (double)theta, &cs, &sn);
-      const bool odd = lane & 1;
+    for (int b2 = 0; b2 < 4; b2 += 2) {
+      // four TMEM loads in flight: blocks b2, b2+1, this warp's 32 heads
+      uint32_t rr[4][16];
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        uint32_t r16[16];
-        sm100::tmem_ld_x16(o_col + 64 * blk + ((uint32_t)(quad * 32) << 16) + 32 * half + 16 * g, r16);
-        sm100::tmem_ld_wait();
+      for (int x = 0; x < 4; ++x)
+        sm100::tmem_ld_x16(o_col + 64 * (b2 + (x >> 1)) + ((uint32_t)(quad * 32) << 16) + 32 * half + 16 * (x & 1),
+                           rr[x]);
+      sm100::tmem_ld_wait();
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int blk = b2 + (x >> 1), g = x & 1;
+        const int c_dim = 128 * blk + quad * 32 + lane;
+        float cs = 1.f, sn = 0.f;
+        if (single && c_dim >= kNope) {
+          cs = S.rope_c[(c_dim - kNope) >> 1];
+          sn = S.rope_s[(c_dim - kNope) >> 1];
+        }
+        const bool odd = lane & 1;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int hl = 16 * g + c;
           const int h = 32 * half + hl;
-          float y = __uint_as_float(r16[c]) * f[hl];
+          float y = __uint_as_float(rr[x][c]) * f[hl];
+          uint16_t bits;
           if (single) {
             const float pv = __shfl_xor_sync(0xffffffffu, y, 1);
             if (c_dim >= kNope) y = odd ? (pv * sn + y * cs) : (y * cs - pv * sn);
-            out[((int64_t)qi * n_heads + h0 + h) * kD + c_dim] = f32_to_bf16_bits(y);
+            bits = f32_to_bf16_bits(y);
           } else {
-            ws_o[(((int64_t)qi * n_splits + split) * n_heads + h0 + h) * kD + c_dim] = __float2half_rn(y);
+            bits = __half_as_ushort(__float2half_rn(y));
           }
+          stage[h * kD + c_dim] = bits;
         }
       }
     }
+    __syncthreads();
+    // 64 rows of 1 KB, 16-byte words: row h = u / 64, word u % 64
+    uint16_t* dst0 = single ? out + ((int64_t)qi * n_heads + h0) * kD
+                            : reinterpret_cast<uint16_t*>(ws_o) + (((int64_t)qi * n_splits + split) * n_heads + h0) * kD;
+#pragma unroll 4
+    for (int u = wt; u < kHg * kD / 8; u += kThreads)
+      reinterpret_cast<uint4*>(dst0)[u] = reinterpret_cast<const uint4*>(stage)[u];
     if (!single && wt < kHg) {
       const int64_t base = ((int64_t)qi * n_splits + split) * n_heads + h0 + wt;
-      ws_ml[base * 2 + 0] = S.mh[wt];
+      ws_ml[base * 2 + 0] = S.mh[wt] * (1.0f / kLog2e);  // natural units
       ws_ml[base * 2 + 1] = S.lh[wt];
     }
   }
@@ -458,53 +569,77 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
 // M = max(sink, m_s), w_s = l_s e^(m_s - M) / (e^(sink - M) + sum l_s
 // e^(m_s - M)), o = sum_s w_s (O_s / l_s) in split order, then the inverse
 // RoPE and a BF16 store.  grid (queries, n_heads / 8), 256 threads: warp =
-// head, lane = 16 dims.
+// head, lane = 16 dims.  The (m, l) of the first 32 splits are read once,
+// one split per lane, and shared by shuffles.
 __global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__ ws_o, const float* __restrict__ ws_ml,
                                                       int n_splits, int n_heads, const float* __restrict__ sink,
                                                       const int32_t* __restrict__ q_pos0, int T, float theta,
                                                       uint16_t* __restrict__ out) {
+  __shared__ float rope_c[kR / 2], rope_s[kR / 2];
   pdl_wait();
   const int qi = blockIdx.x;
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int bs = qi / T, tq = qi % T;
   const int64_t t = (int64_t)q_pos0[bs] + tq;
-  const float sg = sink[h];
-  float M = sg;
-  for (int sp = 0; sp < n_splits; ++sp) M = fmaxf(M, ws_ml[(((int64_t)qi * n_splits + sp) * n_heads + h) * 2]);
-  float den = expf(sg - M);
-  for (int sp = 0; sp < n_splits; ++sp) {
-    const int64_t b2 = (((int64_t)qi * n_splits + sp) * n_heads + h) * 2;
-    const float ms = ws_ml[b2];
-    if (ms != -INFINITY) den += ws_ml[b2 + 1] * expf(ms - M);
+  if (threadIdx.x < kR / 2) {
+    float c, sn;
+    rope_cos_sin(-(double)t, threadIdx.x, kR, (double)theta, &c, &sn);
+    rope_c[threadIdx.x] = c;
+    rope_s[threadIdx.x] = sn;
   }
+  const float sg = sink[h];
+  const int64_t ml0 = ((int64_t)qi * n_splits * n_heads + h) * 2;  // split sp at ml0 + 2 sp n_heads
+  float m_l = -INFINITY, l_l = 0.f;
+  if (lane < n_splits) {
+    m_l = ws_ml[ml0 + (int64_t)2 * lane * n_heads];
+    l_l = ws_ml[ml0 + (int64_t)2 * lane * n_heads + 1];
+  }
+  float M = fmaxf(sg, warp_max(m_l));
+  for (int sp = 32 + lane; sp < n_splits; sp += 32) M = fmaxf(M, ws_ml[ml0 + (int64_t)2 * sp * n_heads]);
+  M = warp_max(M);
+  const float p_l = (m_l == -INFINITY) ? 0.f : l_l * expf(m_l - M);  // split `lane`
+  float part = p_l;
+  for (int sp = 32 + lane; sp < n_splits; sp += 32) {
+    const float ms = ws_ml[ml0 + (int64_t)2 * sp * n_heads];
+    if (ms != -INFINITY) part += ws_ml[ml0 + (int64_t)2 * sp * n_heads + 1] * expf(ms - M);
+  }
+  const float den = expf(sg - M) + warp_sum(part);
   const float inv = den > 0.f ? 1.f / den : 0.f;
+  const float a_l = p_l * inv;  // weight of split `lane` (for lane < 32)
   const int c0 = 16 * lane;
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  const __half* src0 = ws_o + ((int64_t)qi * n_splits * n_heads + h) * kD + c0;
+#pragma unroll 4
   for (int sp = 0; sp < n_splits; ++sp) {
-    const int64_t b2 = (((int64_t)qi * n_splits + sp) * n_heads + h) * 2;
-    const float ms = ws_ml[b2];
-    if (ms == -INFINITY) continue;
-    const float a = ws_ml[b2 + 1] * expf(ms - M) * inv;
-    const uint4* src = reinterpret_cast<const uint4*>(ws_o + (((int64_t)qi * n_splits + sp) * n_heads + h) * kD + c0);
+    float a;
+    if (sp < 32) {
+      a = __shfl_sync(0xffffffffu, a_l, sp);
+    } else {
+      const float ms = ws_ml[ml0 + (int64_t)2 * sp * n_heads];
+      a = ms == -INFINITY ? 0.f : ws_ml[ml0 + (int64_t)2 * sp * n_heads + 1] * expf(ms - M) * inv;
+    }
+    if (a == 0.f) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(src0 + (int64_t)sp * n_heads * kD);
     const uint4 v0 = src[0], v1 = src[1];
-    const __half2* h0 = reinterpret_cast<const __half2*>(&v0);
-    const __half2* h1 = reinterpret_cast<const __half2*>(&v1);
+    const __half2* p0 = reinterpret_cast<const __half2*>(&v0);
+    const __half2* p1 = reinterpret_cast<const __half2*>(&v1);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f0 = __half22float2(h0[e]), f1 = __half22float2(h1[e]);
+      const float2 f0 = __half22float2(p0[e]), f1 = __half22float2(p1[e]);
       acc[2 * e] = fmaf(a, f0.x, acc[2 * e]);
       acc[2 * e + 1] = fmaf(a, f0.y, acc[2 * e + 1]);
       acc[8 + 2 * e] = fmaf(a, f1.x, acc[8 + 2 * e]);
       acc[8 + 2 * e + 1] = fmaf(a, f1.y, acc[8 + 2 * e + 1]);
     }
   }
+  __syncthreads();  // rope table
   if (c0 >= kNope) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      float cs, sn;
-      rope_cos_sin(-(double)t, (c0 - kNope) / 2 + e, kR, (double)theta, &cs, &sn);
+      const int pr = (c0 - kNope) / 2 + e;
+      const float cs = rope_c[pr], sn = rope_s[pr];
       const float x = acc[2 * e], y = acc[2 * e + 1];
       acc[2 * e] = x * cs - y * sn;
       acc[2 * e + 1] = x * sn + y * cs;
@@ -542,10 +677,31 @@ bool attn_tc_supported(const csa_params& p) {
          p.n_heads % kHg == 0 && encode_fn() != nullptr;
 }
 
-int attn_tc_rows_per_split(int total_slots, int T, bool dense) {
+// Rows per split.  Prefill (T > 4): all of a query's slots in one split.
+// Decode: t tiles per split, t minimising  waves x (c + t) + 0.05 x splits,
+// where waves = ceil(CTAs / SMs) (one CTA per SM), c = 0.7 tiles is the
+// fixed cost of a CTA (setup, query load, epilogue) and the last term the
+// merge's share per split.
+int attn_tc_rows_per_split(int total_slots, int nq, int nhg, int T) {
   const int tiles = (total_slots + kRows - 1) / kRows;
-  if (T > 4) return tiles * kRows;           // prefill: one split per query
-  return (dense ? 8 : 1) * kRows;            // decode: fixed split sizes
+  if (T > 4 || tiles <= 1) return (tiles > 1 ? tiles : 1) * kRows;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  int best_t = 1;
+  double best = 1e300;
+  for (int t = 1; t <= tiles; ++t) {
+    const int64_t splits = (tiles + t - 1) / t;
+    const int64_t ctas = (int64_t)nq * nhg * splits;
+    const int64_t waves = (ctas + sms - 1) / sms;
+    const double cost = (double)waves * (0.7 + t) + 0.05 * (double)splits;
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_t = t;
+    }
+  }
+  return best_t * kRows;
 }
 
 size_t attn_tc_smem_bytes() { return sizeof(AttnSmem) + 1024; }
@@ -566,9 +722,9 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
       return cudaErrorInvalidValue;
   }
   const int total = n_sel + p.window;
-  const int rps = attn_tc_rows_per_split(total, T, dense);
-  const int n_splits = (total + rps - 1) / rps;
   const int nhg = p.n_heads / kHg;
+  const int rps = attn_tc_rows_per_split(total, nq, nhg, T);
+  const int n_splits = (total + rps - 1) / rps;
   // workspace: FP16 partials O/l, then (max, sum) per (query, split, head)
   const size_t n_part = (size_t)nq * n_splits * p.n_heads;
   __half* ws_o = reinterpret_cast<__half*>(ws);
@@ -591,7 +747,7 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
 
 size_t attn_tc_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense) {
   const int total = n_sel + p.window;
-  const int rps = attn_tc_rows_per_split(total, T, dense);
+  const int rps = attn_tc_rows_per_split(total, p.B * T, p.n_heads / kHg, T);
   const int n_splits = (total + rps - 1) / rps;
   if (n_splits == 1) return 0;
   const size_t n_part = (size_t)p.B * T * n_splits * p.n_heads;
