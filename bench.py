@@ -10,6 +10,8 @@ hca_dense_attn.  The default workload is the V4-Flash-shaped CSA decode
 
 Timing: W untimed warm-up steps, then exactly K steps between CUDA events on
 the launching stream, bracketed by a barrier and torch.cuda.synchronize().
+In a CSA step the compressor runs on a forked stream beside the index call
+(the two are independent; the attention waits for both).
 The timed loop rotates over several device-resident copies of the workload
 so that the bytes one cycle touches exceed 3x the L2 size: every step reads
 its inputs from HBM, no flush is needed.  Multi-GPU (torchrun): every rank
@@ -289,16 +291,23 @@ def main():
     queries = p.B * w["T"]
     stream = torch.cuda.current_stream()
 
+    side0 = torch.cuda.Stream()
+
     def step(dw, ev=None):
-        dw.compress()
         if p.k > 0:
+            # the compressor runs beside the index call (independent)
+            side0.wait_stream(stream)
+            with torch.cuda.stream(side0):
+                dw.compress(side0)
             if ev is not None:
                 ev[0].record(stream)
             dw.index_topk()
             if ev is not None:
                 ev[1].record(stream)
+            stream.wait_stream(side0)
             dw.sparse_attn()
         else:
+            dw.compress()
             if ev is not None:
                 ev[0].record(stream)
             dw.dense_attn()
@@ -309,16 +318,32 @@ def main():
         step(dws[i % n_copies])
     torch.cuda.synchronize()
 
-    # Each copy's step is captured as three CUDA graphs (compress, the
-    # dominant call, the rest) so that host launch cost does not starve the
-    # device; events between the replays time the dominant call alone.
+    # Each copy's step is captured as CUDA graphs so that host launch cost
+    # does not starve the device; events between the replays time the
+    # dominant call.  CSA: the compressor and the index call are independent
+    # (only the attention reads the new entry), so one graph runs the
+    # compressor on a forked branch concurrently with the index call (the
+    # events around it then time the index call with the compressor
+    # running beside it), a second graph the attention.  HCA: compress, then
+    # the dense attention (dependent).
     graphs = []
     kernels_per_step = None  # counted from the captured graphs when possible
     if not args.no_graph:
         cap = torch.cuda.Stream()
+        side = torch.cuda.Stream()
         cap.wait_stream(stream)
+
+        def fork_compress_index(dw):
+            def run(st):
+                side.wait_stream(st)
+                with torch.cuda.stream(side):
+                    dw.compress(side)
+                dw.index_topk(st)
+                st.wait_stream(side)
+            return run
+
         for dw in dws:
-            phases = [dw.compress, dw.index_topk, dw.sparse_attn] if p.k > 0 else [dw.compress, dw.dense_attn, None]
+            phases = [None, fork_compress_index(dw), dw.sparse_attn] if p.k > 0 else [dw.compress, dw.dense_attn, None]
             parts = []
             with torch.cuda.stream(cap):
                 for fn in phases:

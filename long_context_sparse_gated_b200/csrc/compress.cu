@@ -57,13 +57,37 @@ __global__ void __launch_bounds__(1024) compress_kernel(
   }
   const int n = m + nb;
   const int64_t row0 = (int64_t)bs * S;
+  const int q = threadIdx.x % quads, g = threadIdx.x / quads;
+  const int d0 = q * 4;
+
+  // Latency overlap: the first kPre rows of this thread's token group and
+  // (for the RoPE dims) the rotation of position m*e are fetched / computed
+  // before the gate softmax, which they do not depend on.
+  constexpr int kPre = 4;
+  float pre[kPre][4];
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) {
+    const int i = g + k * G;
+    if (g < G && i < n) {
+      if (i < m)
+        load4<kF32>(a, (row0 + ia0 + i) * d + d0, pre[k]);
+      else
+        load4<kF32>(b, (row0 + ib0 + (i - m)) * d + d0, pre[k]);
+    }
+  }
+  float rc[2] = {1.f, 1.f}, rs_[2] = {0.f, 0.f};
+  if (threadIdx.x < quads && d0 >= d - r) {
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) rope_cos_sin((double)(m * e), (d0 + 2 * pr - (d - r)) >> 1, r, (double)p.rope_theta,
+                                                &rc[pr], &rs_[pr]);
+  }
 
   // 1. softmax over the union of both streams' logits
   float lmax = -INFINITY;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    float g = i < m ? gate[(row0 + ia0 + i) * 2 + 0] : gate[(row0 + ib0 + (i - m)) * 2 + 1];
-    w[i] = g;
-    lmax = fmaxf(lmax, g);
+    const float gl = i < m ? gate[(row0 + ia0 + i) * 2 + 0] : gate[(row0 + ib0 + (i - m)) * 2 + 1];
+    w[i] = gl;
+    lmax = fmaxf(lmax, gl);
   }
   const float gmax = block_max(lmax, red);
   float lsum = 0.f;
@@ -75,12 +99,19 @@ __global__ void __launch_bounds__(1024) compress_kernel(
   const float inv = 1.f / block_sum(lsum, red);  // block_sum syncs: w[] is visible
 
   // 2. weighted merge: group g sums rows i = g, g+G, ...
-  const int q = threadIdx.x % quads, g = threadIdx.x / quads;
-  const int d0 = q * 4;
   float x[4] = {0.f, 0.f, 0.f, 0.f};
   if (g < G) {
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      const int i = g + k * G;
+      if (i < n) {
+        const float wi = w[i] * inv;
+        x[0] = fmaf(wi, pre[k][0], x[0]); x[1] = fmaf(wi, pre[k][1], x[1]);
+        x[2] = fmaf(wi, pre[k][2], x[2]); x[3] = fmaf(wi, pre[k][3], x[3]);
+      }
+    }
 #pragma unroll 4
-    for (int i = g; i < n; i += G) {
+    for (int i = g + kPre * G; i < n; i += G) {
       float v[4];
       if (i < m)
         load4<kF32>(a, (row0 + ia0 + i) * d + d0, v);
@@ -104,17 +135,15 @@ __global__ void __launch_bounds__(1024) compress_kernel(
   // 3. RMSNorm
   float ss = owner ? (y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3]) : 0.f;
   const float tot = block_sum(ss, red);
-  const float rs = 1.f / sqrtf(tot / (float)d + p.eps);
+  const float rsq = 1.f / sqrtf(tot / (float)d + p.eps);
   if (!owner) return;  // no block-wide barrier below this point except via red in FP8 path
 #pragma unroll
-  for (int k = 0; k < 4; ++k) y[k] *= rs * (norm_w ? norm_w[d0 + k] : 1.f);
+  for (int k = 0; k < 4; ++k) y[k] *= rsq * (norm_w ? norm_w[d0 + k] : 1.f);
   // 4. RoPE on the last r dims, pairs (d-r+2j, d-r+2j+1), angle (m*e)*theta^(-2j/r)
   if (d0 >= d - r) {
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
-      const int j = (d0 + 2 * pr - (d - r)) >> 1;
-      float c, s;
-      rope_cos_sin((double)(m * e), j, r, (double)p.rope_theta, &c, &s);
+      const float c = rc[pr], s = rs_[pr];
       const float x0 = y[2 * pr], x1 = y[2 * pr + 1];
       y[2 * pr] = x0 * c - x1 * s;
       y[2 * pr + 1] = x0 * s + x1 * c;

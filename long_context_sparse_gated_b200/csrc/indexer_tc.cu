@@ -13,15 +13,19 @@
 //              rows permuted by a 3-D view, see Stage) and its 512 scale
 //              bytes into a kStages-deep ring; per query (not per tile) the
 //              64x64 B query block and its scales into one of two slots
-//   warp 1     MMA issuer: per query, permutes the query scales into the
-//              32x16 B layout and copies them to TMEM; per tile, copies the
-//              key scales to TMEM (tcgen05.cp) and issues two K=64 MMAs into
-//              one of four TMEM accumulators
-//   warps 2-9  two epilogue warpgroups taking alternate tiles (the epilogue
-//              is the longest stage): tcgen05.ld of the 64 head columns of one entry per
-//              thread, ReLU, weighted head sum, coalesced fp32 store, and
-//              (optionally) the per-query histogram of the scores' top 12
-//              key bits that the top-k selector starts from
+//   warp 1     MMA issuer (one lane): per query, permutes the query scales
+//              into the 32x16 B layout and copies them to TMEM; per tile,
+//              copies the key scales to TMEM (tcgen05.cp), issues two K=64
+//              MMAs into one of four TMEM accumulators and commits them
+//   warps 2-9  two epilogue warpgroups taking alternate tiles: once a
+//              tile's MMAs are complete they release its shared-memory stage
+//              to the producer, tcgen05.ld the 64 head columns of one entry
+//              per thread, ReLU, weighted head sum (four independent partial
+//              sums), fp32 store, and (optionally) count the score's top 12
+//              key bits into the warpgroup's shared-memory histogram of the
+//              current query, which is added to the global per-query
+//              histogram (the top-k selector's starting point) when the
+//              warpgroup moves to another query and at the end
 // Each CTA walks a contiguous range of (query, 128-entry block) tiles, so the
 // key stream it reads is sequential.  Tiles past a query's n_t are skipped.
 //
@@ -67,10 +71,12 @@ struct __align__(1024) QuerySlot {
 
 constexpr int kAcc = 4;         // TMEM accumulators (two per epilogue warpgroup)
 constexpr int kEpiGroups = 2;   // epilogue warpgroups, alternating tiles
+constexpr int kHistBins = 4096; // score histogram bins (top 12 key bits)
 
 struct Smem {
   Stage st[kStages];
   QuerySlot qs[2];
+  uint32_t hist[kEpiGroups][kHistBins];  // per-warpgroup histogram of its current query
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t qfull[2];
@@ -204,46 +210,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    uint32_t it = 0, nq = 0;
-    int cur_q = -1, sl = 0;
-    VisibleCache vc;
-    for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
-      const int qi = c.qi, j = c.j;
-      if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
-      if (qi != cur_q) {
-        // the previous query's slot is free once its MMAs complete
-        if (cur_q >= 0 && lane == 0) sm100::tc_commit(&S.qempty[sl]);
-        sl = nq & 1;
-        int ok = 1;
-        if (lane == 0) ok = sm100::mbar_wait(&S.qfull[sl], (nq >> 1) & 1, abort);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        // query scales: head h's word goes to line h%32, slot h/32
-        QuerySlot& qs = S.qs[sl];
-        uint4 u;
-        u.x = qs.sfq_raw[lane];
-        u.y = qs.sfq_raw[lane + 32];
-        u.z = 0u;
-        u.w = 0u;
-        reinterpret_cast<uint4*>(qs.sfq)[lane] = u;
-        sm100::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
+    // ---------------- MMA issuer (one lane) ----------------
+    if (lane == 0) {
+      uint32_t it = 0, nq = 0;
+      int cur_q = -1, sl = 0;
+      VisibleCache vc;
+      for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
+        const int qi = c.qi, j = c.j;
+        if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
+        if (qi != cur_q) {
+          // the previous query's slot is free once its MMAs complete
+          if (cur_q >= 0) sm100::tc_commit(&S.qempty[sl]);
+          sl = nq & 1;
+          if (!sm100::mbar_wait(&S.qfull[sl], (nq >> 1) & 1, abort)) break;
+          // query scales: head h's word goes to line h%32, slot h/32
+          QuerySlot& qs = S.qs[sl];
+#pragma unroll 4
+          for (int l = 0; l < 32; ++l)
+            reinterpret_cast<uint4*>(qs.sfq)[l] = make_uint4(qs.sfq_raw[l], qs.sfq_raw[l + 32], 0u, 0u);
+          sm100::fence_proxy_async_smem();
           sm100::tc_fence_after();
           sm100::tc_cp_32x128b_warpx4(tmem + kSfbCol + 4 * sl, sm100::smem_desc(sm100::smem_u32(qs.sfq), 0, 128, 0));
+          cur_q = qi;
+          ++nq;
         }
-        cur_q = qi;
-        ++nq;
-      }
-      const int s = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
-      const int acc = it % kAcc;
-      const uint32_t aph = (it / kAcc) & 1;
-      // one lane polls the barriers; the warp follows
-      int ok = 1;
-      if (lane == 0) ok = sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort) && sm100::mbar_wait(&S.full[s], ph, abort);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      if (lane == 0) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        const int acc = it % kAcc;
+        const uint32_t aph = (it / kAcc) & 1;
+        if (!sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort) || !sm100::mbar_wait(&S.full[s], ph, abort)) break;
         sm100::tc_fence_after();
         Stage& st = S.st[s];
         const uint32_t d_col = tmem + acc * kHeads;
@@ -259,11 +254,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
           sm100::mma_mxf4(d_col, adesc, bdesc, sm100::idesc_mxf4(kTileM, kHeads, 2 * kk, 2 * kk), sfa_col,
                           sfb_col, kk);
         }
-        sm100::tc_commit(&S.empty[s]);
+        // completion frees the accumulator's inputs: the epilogue releases
+        // the stage to the producer once it has seen this commit
         sm100::tc_commit(&S.tfull[acc]);
+        ++it;
       }
-      __syncwarp();
-      ++it;
     }
   } else {
     // ---------------- epilogue (warps 2..9: two warpgroups) ----------------
@@ -271,6 +266,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     // TMEM lane 32*quad + lane holds key 4*lane + quad of the tile
     const int key_in_tile = 4 * lane + quad;
+    const int et = threadIdx.x - 64 - 128 * eg;  // 0..127 within the warpgroup
+    uint32_t* sh = S.hist[eg];
+    // add the warpgroup's histogram of query q to the global one and clear it
+    auto flush = [&](int q) {
+      sm100::named_bar_sync(1 + eg, 128);
+      for (int b = et; b < kHistBins; b += 128) {
+        const uint32_t v = sh[b];
+        if (v) {
+          atomicAdd(hist + (int64_t)q * kScoreHistBins + b, v);
+          sh[b] = 0u;
+        }
+      }
+      sm100::named_bar_sync(1 + eg, 128);
+    };
+    if (hist) {
+      for (int b = et; b < kHistBins; b += 128) sh[b] = 0u;
+      sm100::named_bar_sync(1 + eg, 128);
+    }
     uint32_t it = 0;
     int wq = -1;
     float wv[kHeads];
@@ -284,6 +297,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       const int acc = my % kAcc;
       const uint32_t aph = (my / kAcc) & 1;
       if (qi != wq) {  // head weights of this tile's query, kept in registers
+        if (hist && wq >= 0) flush(wq);
         const float4* wp = reinterpret_cast<const float4*>(w + (int64_t)qi * kHeads);
 #pragma unroll
         for (int h4 = 0; h4 < kHeads / 4; ++h4) {
@@ -293,8 +307,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         wq = qi;
       }
       int ok = 1;
-      if (lane == 0) ok = sm100::mbar_wait(&S.tfull[acc], aph, abort);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane == 0) {
+        ok = sm100::mbar_wait(&S.tfull[acc], aph, abort);
+        // the tile's MMAs are complete: its key stage may be refilled
+        if (ok && quad == 0) sm100::mbar_arrive(&S.empty[my % kStages]);
+      }
+      // no break on a failed wait: every warp of the warpgroup keeps walking
+      // the same tiles so that the histogram flushes' named barriers match;
+      // after an abort every wait returns at once and no work is done
+      if (!__shfl_sync(0xffffffffu, ok, 0)) continue;
       sm100::tc_fence_after();
       uint32_t d[64];
       const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + acc * kHeads;
@@ -306,13 +327,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&S.tempty[acc]);
-      float sc = 0.f;
+      // four independent partial sums (every partial sum of these
+      // scores is exact, so the grouping does not change the result)
+      float p4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) sc = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), sc);
+      for (int h = 0; h < kHeads; ++h) p4[h & 3] = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), p4[h & 3]);
+      const float sc = (p4[0] + p4[1]) + (p4[2] + p4[3]);
       const int s_idx = j * kTileM + key_in_tile;
-      if (s_idx < n_t) scores[(int64_t)qi * ld + s_idx] = sc;
-      if (hist) hist_add(hist + (int64_t)qi * kScoreHistBins, score_bin(sc), s_idx < n_t);
+      if (s_idx < n_t) {
+        scores[(int64_t)qi * ld + s_idx] = sc;
+        if (hist) atomicAdd(sh + score_bin(sc), 1u);
+      }
     }
+    if (hist && wq >= 0) flush(wq);
   }
 
   pdl_trigger();
