@@ -217,6 +217,31 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+CONFIG_SEEDS = {"c0": 0, "c1": 1, "c2": 2, "c3": 3, "c4": 4}
+
+
+def rank_seed(config, rank):
+    """Weak scaling: every rank runs the same per-GPU workload shape, drawn
+    from its own seed (no data-path exchange between ranks)."""
+    return CONFIG_SEEDS[config] + 1000 * rank
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of each rank's timings over all ranks of the default
+    process group (every rank must call it, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_value(world, queries_per_rank, ms_per_step):
+    """Whole-job throughput: the queries all ranks processed per second of
+    the slowest rank's step time."""
+    return world * queries_per_rank / (ms_per_step * 1e-3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -278,8 +303,7 @@ def main():
         dist.barrier()
     lib()
 
-    seed_off = 1000 * rank
-    w = synth.config(args.config, seed={"c0": 0, "c1": 1, "c2": 2, "c3": 3, "c4": 4}[args.config] + seed_off)
+    w = synth.config(args.config, seed=rank_seed(args.config, rank))
     step_bytes, idx_bytes = algorithmic_bytes(w)
     n_copies = max(1, int(np.ceil(3 * L2_BYTES / step_bytes)))
     if args.config == "c4":
@@ -443,12 +467,9 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
 
+    kmean = float(np.mean(kern_ms))
     if world > 1:
-        tt = torch.tensor([ms, e2e_ms, float(np.mean(kern_ms))], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, kmean = (float(x) for x in tt.tolist())
-    else:
-        kmean = float(np.mean(kern_ms))
+        ms, e2e_ms, kmean = max_over_ranks([ms, e2e_ms, kmean], "cuda")
     err = int(sum(d.err_bits() for d in dws))
 
     if rank != 0:
@@ -456,7 +477,7 @@ def main():
             dist.destroy_process_group()
         return
     ms_per_step = ms / args.steps
-    value = world * queries / (ms_per_step * 1e-3)
+    value = job_value(world, queries, ms_per_step)
     peak, peak_kind = measured_peaks()
     dom_bytes = idx_bytes if p.k > 0 else step_bytes
     achieved = dom_bytes / (kmean * 1e-3) / 1e9
@@ -478,7 +499,7 @@ def main():
                      "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean},
         "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
                           "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak},
-        "e2e": {"value": world * queries / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_value(world, queries, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clocks,
         "device_err_bits": err,
