@@ -195,6 +195,11 @@ size_t csa_index_topk_workspace_bytes(const csa_params* params, int32_t T,
  * An idx value >= the cache capacity or < -1 is skipped with
  * CSA_DEV_ERR_INDEX.  The window ring must hold every position in
  * [max(0, q_pos0-W+1), q_pos0+T-1] (win.cap >= W + T - 1 suffices).
+ * The slots of a decode query are split over CTAs by a rule that depends on
+ * the shape, the batch and the current device's SM count, so the workspace
+ * size must be queried with the device the call will run on current.
+ * Results are bit-identical run to run; a query's output can differ in its
+ * last bits between batch sizes.
  * ---------------------------------------------------------------------- */
 csa_status csa_sparse_attn(const csa_params* params, const void* q,
                            csa_kv cache, const int32_t* idx, csa_kv win,
