@@ -81,3 +81,15 @@ def test_job_value_is_all_ranks_over_the_slowest_step():
     # 2 ranks x 32 queries in 0.1 ms (the max over ranks) -> 640k queries/s
     assert bench.job_value(2, 32, 0.1) == pytest.approx(640000.0)
     assert bench.job_value(1, 32, 0.1) == pytest.approx(320000.0)
+
+
+def test_attention_flops_closed_form():
+    # HCA: every visible entry plus the window, 4d flops per (head, row)
+    w = synth.config("c3", B=2, L=4096)
+    p = w["params"]
+    n_t = 4096 // p.m
+    assert bench.algorithmic_flops(w) == 2 * p.n_h * (n_t + p.W) * 4 * p.d
+    # CSA: min(k, n_t) selected entries plus the window
+    w = synth.config("c1", B=1, L=8192)
+    p = w["params"]
+    assert bench.algorithmic_flops(w) == p.n_h * (min(p.k, 8192 // p.m) + p.W) * 4 * p.d
