@@ -103,12 +103,16 @@ def algorithmic_flops(w):
 
 
 def launches_per_step(w):
-    """Kernels (and memset nodes) one step enqueues: compress, the indexer's
-    histogram memset + scorer + selector, attention (+ split merge)."""
+    """Kernels one step enqueues (the fallback when the captured graphs'
+    kernel nodes cannot be counted): compress, scorer, selector (plus the
+    chunked candidate pass for rows over 32768 entries), attention (plus the
+    split merge in decode)."""
     p = w["params"]
     n = 1 if w["S"] else 0
     if p.k > 0:
-        n += 3 if w["T"] * p.B <= 4096 else 2
+        hist = w["T"] * p.B <= 4096
+        n_max = int(min(w["Ncap"], ((np.asarray(w["q_pos0"]) + w["T"]) // p.m).max()))
+        n += 2 + (1 if hist and n_max > 32768 else 0)
         n += 2 if w["T"] <= 4 else 1
     else:
         n += 2 if w["T"] <= 4 else 1
