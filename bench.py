@@ -102,6 +102,73 @@ def algorithmic_flops(w):
     return total
 
 
+def index_flops(w):
+    """Lightning Indexer multiply-adds per step (MXFP4 contraction): 2 H_I c_I
+    flops per (query, visible entry)."""
+    p = w["params"]
+    total = 0
+    if p.k <= 0:
+        return 0
+    for b in range(p.B):
+        for tq in range(w["T"]):
+            t = int(w["q_pos0"][b]) + tq
+            total += 2 * p.H_I * p.c_I * min((t + 1) // p.m, w["Ncap"])
+    return total
+
+
+FP4_OVER_BF16 = 4.0  # nominal dense ratio of B200's FP4 and BF16 tensor rates (9 / 2.25 PFLOP/s)
+
+
+def dominant_roofline(w, kmean_ms, idx_bytes, step_bytes, hbm, bf16, traffic):
+    """Roofline entry of the step's dominant call.  hbm = (GB/s, source) and
+    bf16 = (TFLOP/s, source) are the measured peaks.
+
+    CSA decode: the index call streams every visible key once, HBM-bound.
+    CSA prefill: the index call's MXFP4 contraction is tensor-bound (peak:
+    the measured BF16 peak times the nominal FP4:BF16 ratio).  HCA: the dense
+    attention, 4d flops per (head, row), is tensor-bound (BF16 peak; FP16
+    operands run at the BF16 rate)."""
+    p = w["params"]
+    sec = kmean_ms * 1e-3
+    hbm_peak, hbm_src = hbm
+    bf16_peak, bf16_src = bf16
+    dom_bytes = idx_bytes if p.k > 0 else step_bytes
+    hbm_ach = dom_bytes / sec / 1e9
+    if p.k > 0:
+        fl = index_flops(w)
+        fp4_peak = bf16_peak * FP4_OVER_BF16
+        fp4_ach = fl / sec / 1e12
+        if w["T"] <= 4:
+            return {"bound": "hbm", "kernel": "csa_index_topk", "achieved": hbm_ach, "peak": hbm_peak,
+                    "unit": "GB/s", "frac": hbm_ach / hbm_peak, "peak_source": hbm_src, "traffic": traffic,
+                    "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean_ms,
+                    "fp4_tflops": fp4_ach, "fp4_frac": fp4_ach / fp4_peak}
+        return {"bound": "tensor", "kernel": "csa_index_topk", "achieved": fp4_ach, "peak": fp4_peak,
+                "unit": "TFLOP/s", "frac": fp4_ach / fp4_peak,
+                "peak_source": f"{bf16_src} bf16 x {FP4_OVER_BF16:g} (nominal fp4:bf16)", "traffic": traffic,
+                "algorithmic_flops_per_launch": fl, "launch_ms": kmean_ms,
+                "hbm_achieved_gbs": hbm_ach, "hbm_frac": hbm_ach / hbm_peak}
+    fl = algorithmic_flops(w)
+    ach = fl / sec / 1e12
+    return {"bound": "tensor", "kernel": "hca_dense_attn", "achieved": ach, "peak": bf16_peak,
+            "unit": "TFLOP/s", "frac": ach / bf16_peak, "peak_source": bf16_src, "traffic": None,
+            "algorithmic_flops_per_launch": fl, "launch_ms": kmean_ms,
+            "hbm_achieved_gbs": hbm_ach, "hbm_frac": hbm_ach / hbm_peak}
+
+
+def step_roofline_entry(w, ms_per_step, step_bytes, hbm_peak, bf16_peak):
+    """The whole step against both roofs: its algorithmic bytes over the HBM
+    peak, and its two contractions (the indexer's MXFP4 flops, the
+    attention's BF16/FP16 flops) over their tensor peaks, all over the step
+    time."""
+    sec = ms_per_step * 1e-3
+    gbs = step_bytes / sec / 1e9
+    fl_i, fl_a = index_flops(w), algorithmic_flops(w)
+    return {"algorithmic_bytes": step_bytes, "achieved_gbs": gbs, "frac": gbs / hbm_peak,
+            "index_fp4_tflops": fl_i / sec / 1e12, "index_fp4_frac": fl_i / sec / 1e12 / (bf16_peak * FP4_OVER_BF16),
+            "attn_tflops": fl_a / sec / 1e12, "attn_bf16_frac": fl_a / sec / 1e12 / bf16_peak}
+
+
 def launches_per_step(w):
     """Kernels one step enqueues (the fallback when the captured graphs'
     kernel nodes cannot be counted): compress, scorer, selector (plus the
@@ -238,6 +305,38 @@ def oracle_sample(w, n_queries):
     else:
         pipeline.dense_attn(w, comp, qs)
     return time.perf_counter() - t0, len(qs)
+
+
+CPU_SAMPLE = {"c0": 1, "c1": 4, "c2": 1, "c3": 4, "c4": 16}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline_entry(w, config):
+    """The oracle on a bounded sample of the workload (its first queries),
+    with the host threads its numpy/BLAS pool uses, then with one thread."""
+    dt, nq = oracle_sample(w, CPU_SAMPLE[config])
+    entry = {"value": nq / dt, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+             "sample": f"first {nq} queries of the workload (numpy fp64 oracle, {dt:.1f} s)",
+             "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            dt1, nq1 = oracle_sample(w, CPU_SAMPLE[config])
+        entry["value_1_thread"] = nq1 / dt1
+    except Exception:
+        pass
+    return entry
 
 
 def cpu_cores():
@@ -534,24 +633,8 @@ def main():
     ms_per_step = ms / args.steps
     value = job_value(world, queries, ms_per_step)
     peak, peak_kind = measured_peaks()
-    dom_bytes = idx_bytes if p.k > 0 else step_bytes
-    achieved = dom_bytes / (kmean * 1e-3) / 1e9
-    if p.k > 0:
-        # the index call streams every visible key once: HBM-bound
-        roofline = {"bound": "hbm", "kernel": "csa_index_topk", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "peak_source": peak_kind,
-                    "traffic": recorded_traffic(f"csa_index_topk@{args.config}"),
-                    "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean}
-    else:
-        # dense attention: 4d flops per (head, row) over ~d+r+4 bytes per
-        # row shared by n_h heads -> far above the ridge: tensor-bound
-        flops = algorithmic_flops(w)
-        tpeak, tkind = measured_tensor_peak()
-        tach = flops / (kmean * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "kernel": "hca_dense_attn", "achieved": tach, "peak": tpeak,
-                    "unit": "TFLOP/s", "frac": tach / tpeak, "peak_source": tkind, "traffic": None,
-                    "algorithmic_flops_per_launch": flops, "launch_ms": kmean,
-                    "hbm_achieved_gbs": achieved, "hbm_frac": achieved / peak}
+    roofline = dominant_roofline(w, kmean, idx_bytes, step_bytes, (peak, peak_kind), measured_tensor_peak(),
+                                 recorded_traffic(f"csa_index_topk@{args.config}") if p.k > 0 else None)
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -564,18 +647,14 @@ def main():
         "gpu_launches_source": "graph kernel nodes" if kernels_per_step is not None else "static count",
         "graphs": not args.no_graph,
         "roofline": roofline,
-        "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
-                          "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak},
+        "step_roofline": step_roofline_entry(w, ms_per_step, step_bytes, peak, measured_tensor_peak()[0]),
         "e2e": {"value": job_value(world, queries, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clocks,
         "device_err_bits": err,
     }
     if not args.no_cpu_baseline and world == 1:
-        n = {"c0": 1, "c1": 4, "c2": 1, "c3": 4, "c4": 16}[args.config]
-        dt, nq = oracle_sample(w, n)
-        line["cpu_baseline"] = {"value": nq / dt, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
-                                "sample": f"first {nq} queries of the workload (numpy fp64 oracle, {dt:.1f} s)"}
+        line["cpu_baseline"] = cpu_baseline_entry(w, args.config)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -93,3 +93,41 @@ def test_attention_flops_closed_form():
     w = synth.config("c1", B=1, L=8192)
     p = w["params"]
     assert bench.algorithmic_flops(w) == p.n_h * (min(p.k, 8192 // p.m) + p.W) * 4 * p.d
+
+
+def test_index_flops_closed_form():
+    w = synth.config("c1", B=2, L=8192)
+    p = w["params"]
+    n_t = 8192 // p.m
+    assert bench.index_flops(w) == 2 * 2 * p.H_I * p.c_I * n_t
+    assert bench.index_flops(synth.config("c3", B=1, L=4096)) == 0
+
+
+def test_dominant_roofline_binds_the_right_roof():
+    hbm, bf16 = (6451.8, "measured"), (1655.5, "measured")
+    # CSA decode: the index call against HBM
+    w = synth.config("c1", B=2, L=8192)
+    _, idx_bytes = bench.algorithmic_bytes(w)
+    r = bench.dominant_roofline(w, 0.01, idx_bytes, 2 * idx_bytes, hbm, bf16, 123)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 123
+    assert r["achieved"] == pytest.approx(idx_bytes / 1e-5 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6451.8)
+    # CSA prefill: the indexer's MXFP4 contraction against 4x the BF16 peak
+    w = synth.config("c4", B=1, L=1024)
+    r = bench.dominant_roofline(w, 2.0, 1e6, 2e6, hbm, bf16, None)
+    assert r["bound"] == "tensor" and r["peak"] == pytest.approx(4 * 1655.5)
+    assert r["achieved"] == pytest.approx(bench.index_flops(w) / 2e-3 / 1e12)
+    # HCA: the dense attention against the BF16 peak
+    w = synth.config("c3", B=1, L=4096)
+    r = bench.dominant_roofline(w, 0.1, 0, 1e6, hbm, bf16, None)
+    assert r["bound"] == "tensor" and r["peak"] == 1655.5 and r["kernel"] == "hca_dense_attn"
+    assert r["achieved"] == pytest.approx(bench.algorithmic_flops(w) / 1e-4 / 1e12)
+    s = bench.step_roofline_entry(w, 0.2, 1e6, 6451.8, 1655.5)
+    assert s["frac"] == pytest.approx(1e6 / 2e-4 / 1e9 / 6451.8) and s["index_fp4_tflops"] == 0
+
+
+def test_cpu_baseline_entry_reports_threads_and_model():
+    e = bench.cpu_baseline_entry(synth.config("c0"), "c0")
+    assert e["kind"] == "oracle" and e["value"] > 0 and e["cores"] >= 1
+    assert e["nproc"] >= 1 and isinstance(e["cpu_model"], str)
+    assert e.get("value_1_thread", 1.0) > 0
