@@ -212,6 +212,16 @@ def index_scores(q: np.ndarray, w: np.ndarray, k: np.ndarray) -> np.ndarray:
     return np.maximum(dots, 0.0) @ w
 
 
+def bf16_scores(scores: np.ndarray) -> np.ndarray:
+    """Index scores rounded to BF16 (round to nearest even) and widened
+    back: the selector's input in the BF16-score variant (Qiaomu blog
+    FP4量化感知训练 and kwkr.cn notes 4.4: the index scores are quantised
+    from FP32 to BF16 before the top-k selector).  The selection rule is
+    unchanged, so entries whose scores collide after rounding are ranked by
+    index."""
+    return codecs.bf16_decode(codecs.bf16_encode(np.asarray(scores, dtype=np.float64)))
+
+
 def topk_select(scores: np.ndarray, n_t: int, k: int) -> np.ndarray:
     """The min(k, n_t) entries s < n_t ranked by (score descending, s
     ascending), returned in ascending order and padded with -1 to length k."""

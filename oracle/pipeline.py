@@ -102,8 +102,9 @@ def all_queries(w):
     return [(b, tq) for b in range(p.B) for tq in range(w["T"])]
 
 
-def index_topk(w, queries=None, return_scores=False):
-    """csa_index_topk: {(b, tq): int32 [k]} (and the fp64 scores)."""
+def index_topk(w, queries=None, return_scores=False, score_fmt="f32"):
+    """csa_index_topk: {(b, tq): int32 [k]} (and the fp64 scores).
+    score_fmt "bf16" selects on the scores rounded to BF16."""
     p = w["params"]
     queries = all_queries(w) if queries is None else queries
     res, scores = {}, {}
@@ -116,10 +117,26 @@ def index_topk(w, queries=None, return_scores=False):
         k = keys_cache[b][:n_t]
         q, wt = index_query(w, b, tq)
         sc = csa.index_scores(q, wt, k)
+        if score_fmt == "bf16":
+            sc = csa.bf16_scores(sc)
         res[(b, tq)] = csa.topk_select(sc, n_t, p.k)
         if return_scores:
             scores[(b, tq)] = sc
     return (res, scores) if return_scores else res
+
+
+def bf16_score_recall(w, queries):
+    """Recall of the FP32-score top-k by the BF16-score top-k, per query:
+    |selected with BF16 scores  and  selected with FP32 scores| / min(k, n_t)."""
+    p = w["params"]
+    f32 = index_topk(w, queries)
+    b16 = index_topk(w, queries, score_fmt="bf16")
+    out = {}
+    for q in queries:
+        a, b = f32[q], b16[q]
+        n = int((a >= 0).sum())
+        out[q] = len(set(a[a >= 0].tolist()) & set(b[b >= 0].tolist())) / max(n, 1)
+    return out
 
 
 def _query(w, b, tq):

@@ -316,3 +316,26 @@ def test_hca_pipeline_window_and_causality():
             q = w["q"][b, tq].astype(np.float64)
             ref = csa.rope(csa.dense_softmax_with_null_value(q, vals, w["sink"], p.tau), -t, 1e4, 8)
             np.testing.assert_allclose(out[(b, tq)], ref, atol=1e-12)
+
+
+# ---- BF16 index scores (the selector's low-precision variant) -------------
+
+def test_bf16_scores_round_to_nearest_even_like_torch():
+    import torch
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.normal(size=2000) * 37.0, [0.0, 1.0, 1.00390625, 1.01171875, 3.0e-3]])
+    ref = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(csa.bf16_scores(x.astype(np.float32).astype(np.float64)), ref)
+
+
+def test_bf16_topk_ranks_collisions_by_index():
+    # 1 + 2^-9 and 1 + 2^-10 both round to 1.0 in BF16: after rounding the
+    # three entries tie and the lowest indices win
+    sc = np.array([1.0, 1.0 + 2.0 ** -10, 1.0 + 2.0 ** -9, 0.5])
+    assert csa.topk_select(sc, 4, 2).tolist() == [1, 2]
+    assert csa.topk_select(csa.bf16_scores(sc), 4, 2).tolist() == [0, 1]
+
+
+def test_bf16_recall_is_one_when_everything_is_selected():
+    w = synth.config("c1", B=1, L=1024)  # n_t = 256 <= k = 512
+    assert pipeline.bf16_score_recall(w, [(0, 0)]) == {(0, 0): 1.0}
