@@ -291,11 +291,29 @@ def measured_tensor_peak():
         return 1590.0, "fallback"
 
 
-def oracle_sample(w, n_queries):
-    """Time the oracle on the first n_queries queries of the workload."""
+def sample_queries(w, config):
+    """The bounded sample of queries the oracle is timed on, and its
+    description.  Decode: the first few queries.  Prefill: a stratified
+    sample of sequence 0's positions (the oracle's cost grows with the
+    position): the first 16, 16 around t = 2047, the last 16 and 16 seeded
+    uniform others."""
+    p = w["params"]
+    T = w["T"]
+    if T <= 4:
+        n = CPU_SAMPLE[config]
+        return [(b, tq) for b in range(p.B) for tq in range(T)][:n], f"first {n} queries of the workload"
+    pos = set(range(16)) | set(range(max(0, 2040), min(T, 2056))) | set(range(T - 16, T))
+    rest = np.setdiff1d(np.arange(T), np.fromiter(pos, dtype=np.int64))
+    pos |= set(int(x) for x in np.random.default_rng(12345).choice(rest, size=min(16, len(rest)), replace=False))
+    qs = [(0, int(tq)) for tq in sorted(pos)]
+    return qs, (f"{len(qs)} positions of sequence 0: first 16, 16 around t=2047, last 16, 16 seeded uniform")
+
+
+def oracle_sample(w, queries):
+    """Time the oracle on the given queries of the workload."""
     from oracle import pipeline
     p = w["params"]
-    qs = [(b, tq) for b in range(p.B) for tq in range(w["T"])][:n_queries]
+    qs = list(queries)
     seqs = sorted(set(b for b, _ in qs))
     t0 = time.perf_counter()
     comp = pipeline.compress(w, seqs=seqs) if w["S"] else None
@@ -325,14 +343,15 @@ def cpu_model():
 def cpu_baseline_entry(w, config):
     """The oracle on a bounded sample of the workload (its first queries),
     with the host threads its numpy/BLAS pool uses, then with one thread."""
-    dt, nq = oracle_sample(w, CPU_SAMPLE[config])
+    qs, what = sample_queries(w, config)
+    dt, nq = oracle_sample(w, qs)
     entry = {"value": nq / dt, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
-             "sample": f"first {nq} queries of the workload (numpy fp64 oracle, {dt:.1f} s)",
+             "sample": f"{what} (numpy fp64 oracle, {dt:.1f} s)",
              "cpu_model": cpu_model(), "nproc": os.cpu_count()}
     try:
         from threadpoolctl import threadpool_limits
         with threadpool_limits(limits=1):
-            dt1, nq1 = oracle_sample(w, CPU_SAMPLE[config])
+            dt1, nq1 = oracle_sample(w, qs)
         entry["value_1_thread"] = nq1 / dt1
     except Exception:
         pass
@@ -378,12 +397,13 @@ def run_reference(args):
     if rank != 0:
         return
     w = synth.config(args.config)
-    n = {"c0": 1, "c1": 4, "c2": 1, "c3": 4, "c4": 16}[args.config]
+    qs, what = sample_queries(w, args.config)
+    n = len(qs)
     for _ in range(args.warmup and 1):
-        oracle_sample(w, 1)
+        oracle_sample(w, qs[:1])
     times = []
     for _ in range(args.steps):
-        dt, nq = oracle_sample(w, n)
+        dt, nq = oracle_sample(w, qs)
         times.append(dt)
     total = sum(times)
     qps = args.steps * n / total
@@ -393,7 +413,8 @@ def run_reference(args):
             "data": "synthetic", "config": {"workload": CONFIG_NAMES[args.config], "name": args.config,
                                             "sample_queries_per_step": n},
             "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
-                             "sample": f"first {n} queries of the workload per step (oracle: numpy fp64)"},
+                             "sample": f"{what} per step (oracle: numpy fp64)", "cpu_model": cpu_model(),
+                             "nproc": os.cpu_count()},
             "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
