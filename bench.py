@@ -141,6 +141,7 @@ def dominant_roofline(w, kmean_ms, idx_bytes, step_bytes, hbm, bf16, traffic):
         if w["T"] <= 4:
             return {"bound": "hbm", "kernel": "csa_index_topk", "achieved": hbm_ach, "peak": hbm_peak,
                     "unit": "GB/s", "frac": hbm_ach / hbm_peak, "peak_source": hbm_src, "traffic": traffic,
+                    "frac_vs_8tbs_datasheet": hbm_ach / 8000.0,
                     "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean_ms,
                     "fp4_tflops": fp4_ach, "fp4_frac": fp4_ach / fp4_peak}
         return {"bound": "tensor", "kernel": "csa_index_topk", "achieved": fp4_ach, "peak": fp4_peak,

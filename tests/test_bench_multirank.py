@@ -112,6 +112,7 @@ def test_dominant_roofline_binds_the_right_roof():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 123
     assert r["achieved"] == pytest.approx(idx_bytes / 1e-5 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 6451.8)
+    assert r["frac_vs_8tbs_datasheet"] == pytest.approx(r["achieved"] / 8000.0)
     # CSA prefill: the indexer's MXFP4 contraction against 4x the BF16 peak
     w = synth.config("c4", B=1, L=1024)
     r = bench.dominant_roofline(w, 2.0, 1e6, 2e6, hbm, bf16, None)
