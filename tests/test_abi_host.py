@@ -79,3 +79,26 @@ def test_host_validation_codes():
     assert r["ws_bytes"] == 2 * 32768 * 4 + 2 * 4096 * 4  # scores + per-query histograms
     assert r["attn_ws"] > 0
     assert r["name"] == "CSA_ERR_WORKSPACE"
+
+
+def test_plain_c_client_compiles_links_and_validates(tmp_path):
+    """The header is a C99 header: a C program builds against it alone,
+    links libcsa.so and gets the documented status codes."""
+    import shutil
+    from long_context_sparse_gated_b200 import build
+    lib_path = build.build()
+    cc = shutil.which("gcc") or shutil.which("cc")
+    assert cc, "no C compiler"
+    exe = tmp_path / "abi_c_client"
+    libdir = os.path.dirname(lib_path)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "abi_c_client.c"), "-L", libdir, "-l:" + os.path.basename(lib_path),
+                        "-Wl,-rpath," + libdir, "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([str(exe)], capture_output=True, text=True, env=env, timeout=120)
+    assert out.returncode == 0, out.stderr
+    s_null, s_bad, s_align, ws, name = out.stdout.split()
+    assert (int(s_null), int(s_bad), int(s_align)) == (-1, -2, -3)
+    assert int(ws) == 2 * 32768 * 4 + 2 * 4096 * 4
+    assert name == "CSA_ERR_ALIGN"
