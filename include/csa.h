@@ -155,6 +155,48 @@ csa_status hca_compress(const csa_params* params, const void* a, const void* b,
                         int32_t* out_pos, int32_t* err, void* stream);
 
 /* ------------------------------------------------------------------------
+ * csa_index_compress  [kwkr 3.1 (the indexer scores the compressed
+ *                      entries), 3.4 and 4.4 (its QK runs in FP4);
+ *                      Qiaomu FP4量化感知训练]
+ *
+ * Index keys of entries e in [e_begin[b], e_end[b]): the compressor of
+ * csa_compress (gated two-stream merge, RMSNorm, RoPE at position m*e)
+ * run over the idx_dim-dim indexer streams, with RoPE on their last
+ * rope_dims dims (0 <= rope_dims <= idx_dim, a multiple of 4), then
+ * converted to MXFP4 by the OCP MX v1.0 rule: per block of 32 dims the
+ * shared exponent X = floor(log2 max|v|) - 2 (E2M1's largest exponent),
+ * clamped to [-127, 127] (-127 for an all-zero block), stored as the UE8M0
+ * byte X + 127; each element the E2M1 code of v / 2^X, rounded to nearest
+ * even and saturated to +-6.
+ *
+ *   a, b       [B][S][idx_dim] indexer streams (act_fmt), row p - tok_base[b]
+ *   gate       [B][S][2] fp32 logits
+ *   tok_base, e_begin, e_end, max_entries, norm_w ([idx_dim] or NULL): as
+ *              for csa_compress
+ *   k_idx      [B][k_cap][idx_dim/2] MXFP4 key rows (row e written),
+ *   k_idx_sf   [B][k_cap][idx_dim/32] UE8M0 scales
+ * Entries whose tokens fall outside the buffer or whose slot is >= k_cap
+ * are skipped with CSA_DEV_ERR_RANGE.  idx_dim must be 64 or 128.
+ * ---------------------------------------------------------------------- */
+csa_status csa_index_compress(const csa_params* params, const void* a, const void* b,
+                              const float* gate, int64_t S, const int32_t* tok_base,
+                              const int32_t* e_begin, const int32_t* e_end,
+                              int32_t max_entries, int32_t rope_dims, const float* norm_w,
+                              void* k_idx, uint8_t* k_idx_sf, int64_t k_cap, int32_t* err,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
+ * csa_index_quantize  [kwkr 3.4: the indexer QK runs directly in FP4]
+ *
+ * n_rows rows of idx_dim values x [n_rows][idx_dim] (act_fmt) -> MXFP4
+ * rows out [n_rows][idx_dim/2] and scales out_sf [n_rows][idx_dim/32], by
+ * the OCP MX rule of csa_index_compress.  For the index queries of a call,
+ * n_rows = B * T * n_idx_heads.
+ * ---------------------------------------------------------------------- */
+csa_status csa_index_quantize(const csa_params* params, const void* x, int64_t n_rows,
+                              void* out, uint8_t* out_sf, void* stream);
+
+/* ------------------------------------------------------------------------
  * csa_index_topk  [Qiaomu 混合注意力机制, FP4量化感知训练; kwkr 3.4, 4.4;
  *                  PACMAN 3.1]
  *
@@ -195,11 +237,16 @@ size_t csa_index_topk_workspace_bytes(const csa_params* params, int32_t T,
  * An idx value >= the cache capacity or < -1 is skipped with
  * CSA_DEV_ERR_INDEX.  The window ring must hold every position in
  * [max(0, q_pos0-W+1), q_pos0+T-1] (win.cap >= W + T - 1 suffices).
- * The slots of a decode query are split over CTAs by a rule that depends on
- * the shape, the batch and the current device's SM count, so the workspace
- * size must be queried with the device the call will run on current.
- * Results are bit-identical run to run; a query's output can differ in its
- * last bits between batch sizes.
+ * Batch invariance: a query's slots are split over CTAs by a rule that
+ * depends only on its own slot count, n_heads and T -- never on the batch,
+ * the other sequences or the device -- and split partials are merged in a
+ * fixed order, so a query's output is bit-identical run to run and whatever
+ * batch it is in (for the same T).
+ * Input range: FP8 row scales must lie in [2^-90, 2^90] (rows outside are
+ * skipped with CSA_DEV_ERR_RANGE); RoPE dims and queries may be any finite
+ * BF16.  Logits tau*q.v are formed exactly up to fp32 rounding and must be
+ * finite in fp32 (a row with a non-finite logit is skipped with
+ * CSA_DEV_ERR_RANGE).
  * ---------------------------------------------------------------------- */
 csa_status csa_sparse_attn(const csa_params* params, const void* q,
                            csa_kv cache, const int32_t* idx, csa_kv win,
@@ -235,10 +282,15 @@ size_t hca_dense_attn_workspace_bytes(const csa_params* params, int32_t T,
  * library until the process exits).  Returns CSA_ERR_WORKSPACE, launching
  * nothing, when csa_index_topk_workspace_bytes(params, T, n_max) exceeds
  * 16 MiB.  It allocates nothing (no cudaMalloc/cudaFree, no allocating
- * library call).  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture.  Every call shares the one array: calls
- * whose work overlaps on the GPU race on it.
+ * library call) itself, but the array lives in a library module that the
+ * CUDA runtime loads on a device lazily: the first call on a device loads it
+ * there, which reserves the 16 MiB (an out-of-memory failure then returns
+ * CSA_ERR_LAUNCH), and looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current).  Make that first call
+ * during set-up, before any allocation-free region and before any stream
+ * capture.  If the device's context is destroyed (cudaDeviceReset), the next
+ * call loads the module again and looks the address up anew.  Every call
+ * shares the one array: calls whose work overlaps on the GPU race on it.
  * ---------------------------------------------------------------------- */
 csa_status csa_index_topk_noalloc(const csa_params* params, const void* q_idx,
                                   const uint8_t* q_idx_sf, const float* w,

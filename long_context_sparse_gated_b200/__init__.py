@@ -20,7 +20,8 @@ __all__ = [
     "CsaParams", "CsaKv", "CsaError", "lib", "make_params",
     "csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn",
     "csa_index_topk_workspace_bytes", "csa_sparse_attn_workspace_bytes",
-    "hca_dense_attn_workspace_bytes", "csa_index_topk_noalloc", "KV_F32", "KV_FP8_BF16", "IDX_F32", "IDX_MXFP4",
+    "hca_dense_attn_workspace_bytes", "csa_index_topk_noalloc", "csa_index_compress", "csa_index_quantize",
+    "KV_F32", "KV_FP8_BF16", "IDX_F32", "IDX_MXFP4",
     "ACT_F32", "ACT_BF16", "DEV_ERR_INDEX", "DEV_ERR_RANGE",
 ]
 
@@ -38,7 +39,7 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID", -2: "CSA_ERR_UNSUPPORTED", -3: "CS
 EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_index_topk_workspace_bytes",
            "csa_sparse_attn", "csa_sparse_attn_workspace_bytes", "hca_dense_attn",
            "hca_dense_attn_workspace_bytes", "csa_status_string", "csa_last_error_string",
-           "csa_index_topk_noalloc"]
+           "csa_index_topk_noalloc", "csa_index_compress", "csa_index_quantize"]
 
 
 class CsaError(RuntimeError):
@@ -90,6 +91,10 @@ def lib(path: str | None = None):
     L.hca_dense_attn.argtypes = [_P, _V, CsaKv, CsaKv, _V, _V, _I32, _I32, _V, _V, _SZ, _V, _V]
     L.hca_dense_attn_workspace_bytes.argtypes = [_P, _I32, _I32]
     L.hca_dense_attn_workspace_bytes.restype = _SZ
+    L.csa_index_compress.argtypes = [_P, _V, _V, _V, _I64, _V, _V, _V, _I32, _I32, _V, _V, _V, _I64, _V, _V]
+    L.csa_index_compress.restype = _I32
+    L.csa_index_quantize.argtypes = [_P, _V, _I64, _V, _V, _V]
+    L.csa_index_quantize.restype = _I32
     L.csa_status_string.argtypes = [_I32]
     L.csa_status_string.restype = ctypes.c_char_p
     L.csa_last_error_string.argtypes = []
@@ -156,6 +161,25 @@ def hca_compress(params, a, b, gate, tok_base, e_begin, e_end, max_entries, out_
                  out_pos=None, norm_w=None, err=None, stream=None):
     csa_compress(params, a, b, gate, tok_base, e_begin, e_end, max_entries, out_rows, out_scale,
                  out_pos, norm_w, err, stream, _name="hca_compress")
+
+
+def csa_index_compress(params, a, b, gate, tok_base, e_begin, e_end, max_entries, rope_dims, k_idx, k_idx_sf,
+                       norm_w=None, err=None, stream=None):
+    """Index keys of entries [e_begin[b], e_end[b]) from the indexer streams
+    ``a``/``b`` ([B, S, idx_dim]) into ``k_idx`` ([B, k_cap, idx_dim/2]) and
+    ``k_idx_sf`` ([B, k_cap, idx_dim/32])."""
+    st = lib().csa_index_compress(ctypes.byref(params), _ptr(a), _ptr(b), _ptr(gate), a.shape[1], _ptr(tok_base),
+                                  _ptr(e_begin), _ptr(e_end), int(max_entries), int(rope_dims), _ptr(norm_w),
+                                  _ptr(k_idx), _ptr(k_idx_sf), k_idx.shape[1], _ptr(err), _stream(stream))
+    _check("csa_index_compress", st)
+
+
+def csa_index_quantize(params, x, out, out_sf, stream=None):
+    """Rows of ``x`` ([..., idx_dim]) to MXFP4 ``out`` ([..., idx_dim/2]) and
+    ``out_sf`` ([..., idx_dim/32])."""
+    n_rows = x.numel() // params.idx_dim
+    st = lib().csa_index_quantize(ctypes.byref(params), _ptr(x), n_rows, _ptr(out), _ptr(out_sf), _stream(stream))
+    _check("csa_index_quantize", st)
 
 
 def csa_index_topk_workspace_bytes(params, T, n_max):

@@ -2,7 +2,6 @@
 // allocates, synchronises or keeps state; every call only enqueues kernels
 // on the caller's stream.
 #include <cuda_runtime.h>
-#include <stdlib.h>
 
 #include "csa.h"
 #include "kernels.h"
@@ -42,13 +41,6 @@ csa_status check_kv(const csa_params* p, const csa_kv& kv) {
   return CSA_OK;
 }
 
-// CSA_INDEXER=simt selects the CUDA-core indexer instead of the tensor-core
-// one (a diagnostic switch: both compute the same scores).
-bool simt_indexer_requested() {
-  const char* v = getenv("CSA_INDEXER");
-  return v && v[0] == 's';
-}
-
 thread_local const char* g_last_error = "no error";
 
 csa_status launched(cudaError_t e) {
@@ -56,6 +48,14 @@ csa_status launched(cudaError_t e) {
   g_last_error = cudaGetErrorString(e);
   return CSA_ERR_LAUNCH;
 }
+
+}  // namespace
+
+namespace csa {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace csa
+
+namespace {
 
 csa_status compress_impl(const csa_params* p, const void* a, const void* b, const float* gate,
                          int64_t S, const int32_t* tok_base, const int32_t* e_begin,
@@ -110,6 +110,40 @@ csa_status hca_compress(const csa_params* p, const void* a, const void* b, const
                        out_pos, err, stream);
 }
 
+csa_status csa_index_compress(const csa_params* p, const void* a, const void* b, const float* gate, int64_t S,
+                              const int32_t* tok_base, const int32_t* e_begin, const int32_t* e_end,
+                              int32_t max_entries, int32_t rope_dims, const float* norm_w, void* k_idx,
+                              uint8_t* k_idx_sf, int64_t k_cap, int32_t* err, void* stream) {
+  if (!p) return CSA_ERR_INVALID;
+  if (p->B < 1 || p->m < 1 || max_entries < 0 || S < 1 || k_cap < 1) return CSA_ERR_INVALID;
+  if (p->m > 256) return CSA_ERR_UNSUPPORTED;
+  if (p->idx_dim != 64 && p->idx_dim != 128) return CSA_ERR_UNSUPPORTED;
+  if (rope_dims < 0 || rope_dims > p->idx_dim || (rope_dims & 3)) return CSA_ERR_UNSUPPORTED;
+  if (p->act_fmt != CSA_ACT_F32 && p->act_fmt != CSA_ACT_BF16) return CSA_ERR_UNSUPPORTED;
+  if (!(p->eps >= 0.f) || !(p->rope_theta > 0.f)) return CSA_ERR_INVALID;
+  if (!a || !b || !gate || !tok_base || !e_begin || !e_end || !k_idx || !k_idx_sf) return CSA_ERR_INVALID;
+  for (const void* ptr : {a, b, (const void*)gate, (const void*)tok_base, (const void*)e_begin,
+                          (const void*)e_end, (const void*)k_idx, (const void*)k_idx_sf})
+    if (!aligned16(ptr)) return CSA_ERR_ALIGN;
+  if (norm_w && !aligned16(norm_w)) return CSA_ERR_ALIGN;
+  if (max_entries == 0) return CSA_OK;
+  return launched(csa::launch_index_compress(*p, rope_dims, a, b, gate, S, tok_base, e_begin, e_end, max_entries,
+                                             norm_w, k_idx, k_idx_sf, k_cap, err,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+csa_status csa_index_quantize(const csa_params* p, const void* x, int64_t n_rows, void* out, uint8_t* out_sf,
+                              void* stream) {
+  if (!p || n_rows < 0) return CSA_ERR_INVALID;
+  if (p->idx_dim != 64 && p->idx_dim != 128) return CSA_ERR_UNSUPPORTED;
+  if (p->act_fmt != CSA_ACT_F32 && p->act_fmt != CSA_ACT_BF16) return CSA_ERR_UNSUPPORTED;
+  if (n_rows == 0) return CSA_OK;
+  if (!x || !out || !out_sf) return CSA_ERR_INVALID;
+  for (const void* ptr : {x, (const void*)out, (const void*)out_sf})
+    if (!aligned16(ptr)) return CSA_ERR_ALIGN;
+  return launched(csa::launch_index_quantize(*p, x, n_rows, out, out_sf, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t csa_index_topk_workspace_bytes(const csa_params* p, int32_t T, int32_t n_max) {
   if (!p || T < 1 || n_max < 0 || p->B < 1) return 0;
   return index_ws_bytes(p, T, n_max);
@@ -139,8 +173,7 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* scores = reinterpret_cast<float*>(ws);
   const int ld = csa::topk_scores_ld(n_max);
-  const bool tc = csa::index_scores_tc_supported(*p, k_cap, q_idx, q_idx_sf, k_idx, k_idx_sf) &&
-                  !simt_indexer_requested();
+  const bool tc = csa::index_scores_tc_supported(*p, k_cap, q_idx, q_idx_sf, k_idx, k_idx_sf);
   uint32_t* hist = nullptr;
   if (tc && csa::topk_use_hist(p->B * T) && n_max > p->topk) {
     hist = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + scores_bytes(p, T, n_max));

@@ -14,8 +14,6 @@
 // head group), runs an online softmax over 32-row tiles and either writes
 // the final output (single split) or an unnormalised partial (O, max,
 // sum) that attn_merge combines in split order.
-#include <stdlib.h>
-
 #include "common.cuh"
 #include "kernels.h"
 
@@ -54,7 +52,13 @@ __global__ void __launch_bounds__(256) attn_split_simt(
   const int64_t n_t = (t + 1) / p.m;
   const int h0 = hg * kHeadGroup;
   const int nh = min(kHeadGroup, p.n_heads - h0);
-  const int total = n_sel + W;
+  // this query's own slots (CSA: the k selected entries; HCA: its n_t
+  // visible ones), then its window; a query with one split is finalised
+  // here, one with several writes partials for attn_merge
+  const int own_sel = kDense ? (int)min((int64_t)n_sel, n_t) : n_sel;
+  const int total = own_sel + W;
+  const int own_splits = (total + rows_per_split - 1) / rows_per_split;
+  if (split >= own_splits) return;
   const int sb = split * rows_per_split;
   const int se = min(total, sb + rows_per_split);
 
@@ -90,7 +94,7 @@ __global__ void __launch_bounds__(256) attn_split_simt(
       int src = 0;
       int64_t row = 0;
       if (slot < se) {
-        if (slot < n_sel) {
+        if (slot < own_sel) {
           if (kDense) {
             if (slot < n_t && slot < cache.cap) { src = 1; row = slot; }
           } else {
@@ -102,7 +106,7 @@ __global__ void __launch_bounds__(256) attn_split_simt(
             }
           }
         } else {
-          const int64_t pos = t - W + 1 + (slot - n_sel);
+          const int64_t pos = t - W + 1 + (slot - own_sel);
           if (pos >= 0) { src = 2; row = pos % win.cap; }
         }
       }
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(256) attn_split_simt(
     __syncthreads();
   }
 
-  if (n_splits > 1) {
+  if (own_splits > 1) {
     const int64_t base = ((int64_t)qi * n_splits + split) * p.n_heads + h0;
 #pragma unroll
     for (int h = 0; h < kHeadGroup; ++h) {
@@ -223,20 +227,24 @@ template <bool kActF32>
 __global__ void __launch_bounds__(256) attn_merge(const csa_params p, const float* __restrict__ ws_o,
                                                   const float* __restrict__ ws_ml, int n_splits,
                                                   const float* __restrict__ sink,
-                                                  const int32_t* __restrict__ q_pos0, int T,
-                                                  void* __restrict__ out) {
+                                                  const int32_t* __restrict__ q_pos0, int T, int n_sel,
+                                                  int dense, int rows_per_split, void* __restrict__ out) {
   const int d = p.d, r = p.r, nth = blockDim.x;
   const int qi = blockIdx.x, h = blockIdx.y;
   const int bs = qi / T, tq = qi % T;
   const int64_t t = (int64_t)q_pos0[bs] + tq;
+  // the query's own split count; n_splits is only the workspace stride
+  const int own_sel = dense ? (int)min((int64_t)n_sel, (t + 1) / p.m) : n_sel;
+  const int own_splits = (own_sel + p.window + rows_per_split - 1) / rows_per_split;
+  if (own_splits <= 1) return;  // finalised by the split kernel
   const float sg = sink[h];
   float Ms = sg;
-  for (int s = 0; s < n_splits; ++s)
+  for (int s = 0; s < own_splits; ++s)
     Ms = fmaxf(Ms, ws_ml[(((int64_t)qi * n_splits + s) * p.n_heads + h) * 2]);
   float den = (Ms == -INFINITY) ? 0.f : expf(sg - Ms);
   const int c0 = threadIdx.x, c1 = threadIdx.x + nth;
   float y0 = 0.f, y1 = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
+  for (int s = 0; s < own_splits; ++s) {
     const int64_t base = ((int64_t)qi * n_splits + s) * p.n_heads + h;
     const float M = ws_ml[base * 2], L = ws_ml[base * 2 + 1];
     if (M == -INFINITY) continue;
@@ -298,25 +306,24 @@ static cudaError_t launch_attn_t(const csa_params& p, const void* q, const csa_k
   kfn<<<grid, p.d / 2, smem, st>>>(p, q, rc, idx, rw, sink, q_pos0, T, n_sel, rps, n_splits, out, ws_o, ws_ml, err);
   e = cudaGetLastError();
   if (e != cudaSuccess || n_splits == 1) return e;
-  return launch_attn_merge(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out, st);
+  return launch_attn_merge(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, n_sel, kDense, rps, out, st);
 }
 
 cudaError_t launch_attn_merge(const csa_params& p, const float* ws_o, const float* ws_ml, int n_splits,
-                              const float* sink, const int32_t* q_pos0, int T, void* out, cudaStream_t st) {
+                              const float* sink, const int32_t* q_pos0, int T, int n_sel, bool dense,
+                              int rows_per_split, void* out, cudaStream_t st) {
   if (p.act_fmt == CSA_ACT_F32)
-    attn_merge<true><<<dim3(p.B * T, p.n_heads), p.d / 2, 0, st>>>(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out);
+    attn_merge<true><<<dim3(p.B * T, p.n_heads), p.d / 2, 0, st>>>(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, n_sel,
+                                                                   dense ? 1 : 0, rows_per_split, out);
   else
-    attn_merge<false><<<dim3(p.B * T, p.n_heads), p.d / 2, 0, st>>>(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, out);
+    attn_merge<false><<<dim3(p.B * T, p.n_heads), p.d / 2, 0, st>>>(p, ws_o, ws_ml, n_splits, sink, q_pos0, T, n_sel,
+                                                                    dense ? 1 : 0, rows_per_split, out);
   return cudaGetLastError();
 }
 
-// CSA_ATTN=simt selects the CUDA-core attention (a diagnostic switch).
-static bool simt_attn_requested() {
-  const char* v = getenv("CSA_ATTN");
-  return v && v[0] == 's';
-}
-
-static bool use_tc(const csa_params& p) { return attn_tc_supported(p) && !simt_attn_requested(); }
+// The tensor-core kernel serves the FP8/BF16 layout at d = 512 with whole
+// 64-head groups; every other shape and format runs on CUDA cores.
+static bool use_tc(const csa_params& p) { return attn_tc_supported(p); }
 
 static size_t attn_simt_workspace_bytes(const csa_params& p, int T, int n_sel) {
   const int total = n_sel + p.window;

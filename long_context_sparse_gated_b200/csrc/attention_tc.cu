@@ -11,31 +11,42 @@
 //   resolve   128 threads map the tile's slots to cache / window rows
 //   gather    the same threads each issue one 576-byte bulk copy (TMA
 //             engine, no tensor map) of their row into a staging area and
-//             load the row's scale; while the copies are in flight the
-//             BF16 query (TMA) is converted to FP16 in place; then the
-//             rows are read from the staging area, converted to FP16 and
-//             stored as a
-//             128-row x 512-dim K-major tile (128-byte swizzle).  E4M3 codes
-//             are exact in FP16; the RoPE dims are stored divided by the row
-//             scale s_j, so that  s_j * (V'_j . q) = v_j . q  and one
-//             accumulator holds a whole logit.
+//             load the row's scale; meanwhile the BF16 query (TMA) arrives
+//             and its amax is taken
+//   convert   the rows are read from the staging area, converted to FP16
+//             and stored as a 128-row x 512-dim K-major tile V' (128-byte
+//             swizzle); the query is converted in place to FP16 times 2^-e
+//             (e from its amax, so that it fits FP16 whatever its BF16
+//             range; 2^e joins the logit factor).
 //   S^T       tcgen05.mma kind::f16 (FP16 A/B, FP32 accumulate):
-//             S^T[j, h] = sum_c V'[j, c] Q[h, c]
+//             S^T[j, h] = sum_c V'[j, c] Q'[h, c]
 //             (M = 128 rows, N = 64 heads, K = 512) into TMEM, 32
-//             back-to-back MMAs from precomputed descriptors
-//   softmax   per row thread: z = tau * s_j * S^T; per-head tile maxima and
-//             sums by warp-transposed shuffles; the running max is raised
-//             lazily (only when a tile exceeds it by > 8), so O is rarely
-//             rescaled; P' = exp(z - m_h) * s_j in FP16, stored MN-major
-//             (each row thread writes its 32 heads as four 16-byte words)
+//             back-to-back MMAs from precomputed descriptors, plus 4 more
+//             that add the FP16 rounding residue of the scaled RoPE dims
+//             (hi + lo parts), so every logit is exact up to fp32 rounding
+//   softmax   per row thread: z = tau * c_j * 2^e * S^T (base 2); per-head
+//             maxima of u = z + log2 c_j and sums by warp-transposed
+//             shuffles; the running max of u is raised lazily (only when a
+//             tile exceeds it by > 11.5), so O is rarely rescaled;
+//             P' = exp2(u - m_h) in FP16 (<= 2^11.5 whatever the row's
+//             scale), stored MN-major; the denominator gets P' / c_j
 //   O^T       tcgen05.mma: O^T[c, h] += sum_j V'[j, c] P'[j, h]
 //             (A = V'^T, the same tile read MN-major; B = P' MN-major;
 //             M = 128 dims x 4 blocks, N = 64 heads, K = 128 rows)
 //   epilogue  normalise (with the sink term when the split is the whole
 //             row set), inverse RoPE, then the 64 x 512 result is staged in
 //             shared memory and written with coalesced 16-byte stores: the
-//             BF16 output, or with several splits the FP16 partial O/l and
-//             (m, l) that attn_merge_f16 combines in split order.
+//             BF16 output, or with several splits the fp32 partial O/l and
+//             (m, l) that attn_merge_f32 combines in split order.
+//
+// Range.  Row j is stored as V'_j = v_j / c_j with c_j = s_j * 2^-k_j: the
+// E4M3 codes times 2^k_j (exact) and the BF16 RoPE dims times 2^k_j / s_j,
+// where k_j <= 0 is the smallest shift that keeps the RoPE dims below 2^15
+// (k_j = 0 unless they exceed about 2^14 s_j).  So every FP16 operand is in
+// range for any finite row scale in [2^-90, 2^90] and any finite BF16 RoPE
+// dims and query; the logit and the output accumulate in fp32.  Rows whose
+// scale is outside that range, and logits that are not finite in fp32, are
+// dropped with CSA_DEV_ERR_RANGE.
 //
 // 8 warps (two per TMEM lane quadrant) gather, run the softmax and the
 // epilogue; thread 0 also issues the query TMA and the MMAs between block
@@ -74,8 +85,14 @@ struct __align__(1024) AttnSmem {
   uint8_t p[kRows * 128];     // P' MN-major: [128 rows][64 heads] FP16, 128B swizzle
   uint8_t q[8][kHg * 128];    // 8 K-chunks: [64 heads][128 B]
   float scale[kRows];
-  float inv_scale[kRows];
+  float code_mul[kRows];      // 2^k_j: factor of the row's E4M3 codes in V'
+  float rope_mul[kRows];      // 2^k_j / s_j: factor of its RoPE dims in V'
+  float row_f[kRows];         // tau * log2(e) * c_j  (c_j = s_j 2^-k_j)
+  float row_lc[kRows];        // log2 c_j
+  float row_ic[kRows];        // 1 / c_j
   int live[kRows];            // row takes part (non-empty slot with a valid scale)
+  uint32_t qamax[kHg];        // fp32 bits of each head's largest query magnitude
+  float qg[kHg];              // 2^e_h: Q'_h = Q_h 2^-e_h
   float red[8][64];
   float mh[kHg], lh[kHg], alpha[kHg];
   float rope_c[kR / 2], rope_s[kR / 2];  // inverse-RoPE rotation of this query
@@ -129,10 +146,42 @@ __device__ __forceinline__ uint4 bf16x8_scale_to_f16(const uint4& in, float s) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// 8 BF16 -> 8 FP16 (round to nearest; queries are RMS-normalised, far
-// inside the FP16 range)
-__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4& in) {
-  return bf16x8_scale_to_f16(in, 1.0f);
+// 8 BF16 values times s as FP16 hi + lo pairs: hi = fp16(x), lo =
+// fp16(x - hi), so that hi + lo carries x to about 22 bits.
+__device__ __forceinline__ void bf16x8_scale_to_f16_hilo(const uint4& in, float s, uint4& hi, uint4& lo) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = bf16_bits_to_f32(w[i]) * s, b = bf16_bits_to_f32(w[i] >> 16) * s;
+    const __half2 hh = __floats2half2_rn(a, b);
+    const float2 hf = __half22float2(hh);
+    const __half2 ll = __floats2half2_rn(a - hf.x, b - hf.y);
+    h[i] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[i] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Largest-magnitude bits of the 8 BF16 values in a 16-byte word (sign
+// cleared; as integers these order like the magnitudes).
+__device__ __forceinline__ uint32_t bf16x8_amax_bits(const uint4& in) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  return m;
+}
+
+// Shift k <= 0 of row j: with R the row's largest RoPE magnitude (BF16
+// bits) and s its scale, R * 2^k / s < 2^15 for k = min(0, 14 + e_s - e_R)
+// (e = unbiased exponent: R < 2^(e_R+1), s >= 2^e_s).
+__device__ __forceinline__ int row_shift(float s, uint32_t rbits) {
+  if (rbits == 0u) return 0;
+  const int e_s = (int)((__float_as_uint(s) >> 23) & 0xFFu) - 127;
+  const int e_r = (int)((rbits >> 7) & 0xFFu) - 127;
+  return min(0, 14 + e_s - e_r);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -192,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     const float* __restrict__ win_scale, int64_t win_cap, const int32_t* __restrict__ idx, int topk,
     const int32_t* __restrict__ q_pos0, int T, int m, int W, int n_sel, int n_heads, float tau,
     float theta, const float* __restrict__ sink, int rows_per_split, int n_splits, uint16_t* __restrict__ out,
-    __half* __restrict__ ws_o, float* __restrict__ ws_ml, int32_t* __restrict__ err) {
+    float* __restrict__ ws_o, float* __restrict__ ws_ml, int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& S = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -203,11 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   const int qi = blockIdx.x, split = blockIdx.y, hg = blockIdx.z;
   const int bs = qi / T, tq = qi % T;
   const int h0 = hg * kHg;
-  const int total = n_sel + W;
-  const int sb = split * rows_per_split;
-  const int se = min(total, sb + rows_per_split);
-  const int n_tiles = (se - sb + kRows - 1) / kRows;
-  const bool single = n_splits == 1;
   volatile int* abort = &S.abort;
   const bool issuer = threadIdx.x == 0;
 
@@ -220,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     sm100::fence_mbar_init();
   }
   if (threadIdx.x < kHg) {
+    S.qamax[threadIdx.x] = 0u;
     S.mh[threadIdx.x] = -INFINITY;
     S.lh[threadIdx.x] = 0.f;
   }
@@ -233,6 +278,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   pdl_wait();  // inputs may come from the previous kernel on the stream
   const int64_t t = (int64_t)q_pos0[bs] + tq;
   const int64_t n_t = (t + 1) / m;
+  // this query's own slots: its entries (CSA: the k selected; HCA: its n_t
+  // visible ones), then its window; split boundaries depend on nothing else
+  const int own_sel = kDense ? (int)min((int64_t)n_sel, n_t) : n_sel;
+  const int total = own_sel + W;
+  const int own_splits = (total + rows_per_split - 1) / rows_per_split;
+  const bool single = own_splits == 1;
+  const int sb = split * rows_per_split;
+  const int se = min(total, sb + rows_per_split);
+  const int n_tiles = se > sb ? (se - sb + kRows - 1) / kRows : 0;
   const uint32_t tmem = S.tmem_base;
   const uint32_t s_col = tmem;         // S^T: 64 columns
   const uint32_t o_col = tmem + 64;    // O^T block b: columns 64 + 64 b
@@ -257,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   const uint64_t dQ = sm100::smem_desc(sm100::smem_u32(S.q[0]), 16, 1024, 2);
   const uint64_t dVt = sm100::smem_desc(sm100::smem_u32(S.v[0]), kRows * 128, 1024, 2);
   const uint64_t dP = sm100::smem_desc(sm100::smem_u32(S.p), kRows * 128, 1024, 2);
+  const uint64_t dPk = sm100::smem_desc(sm100::smem_u32(S.p), 16, 1024, 2);  // P' buffer read K-major (RoPE lo parts)
 
   // Row of this thread (wt < kRows) in the current tile, resolved one tile
   // ahead: while tile i is computed, tile i+1's rows are resolved, their
@@ -265,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   int64_t my_off = -1;
   float my_sc = 1.f;
   if (wt < kRows && n_tiles > 0) {
-    my_src = resolve_slot<kDense>(sb + wt, se, n_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap, err, &my_off);
+    my_src = resolve_slot<kDense>(sb + wt, se, own_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap, err, &my_off);
     if (my_src == 1) my_sc = cache_scale[my_off];
     if (my_src == 2) my_sc = win_scale[my_off];
   }
@@ -290,27 +345,58 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     if (wt < kRows) {
       float sc = my_sc;
       int live = my_src != 0;
-      if (!(sc > 0.f) || !(sc < INFINITY)) {  // scales are positive and finite by construction
+      if (!(sc >= 0x1p-90f) || !(sc <= 0x1p90f)) {  // outside the supported scale range
         if (my_src) raise_err(err, CSA_DEV_ERR_RANGE);
         live = 0;  // the row is dropped (zeroed below)
         sc = 1.f;
       }
       S.live[wt] = live;
       S.scale[wt] = sc;
-      S.inv_scale[wt] = 1.f / sc;
     }
     if (i == 0) {
-      // queries: BF16 (TMA) -> FP16 in place, same swizzled positions
+      // each head's largest BF16 query magnitude (converted after the
+      // barrier).  Word e of the query tile is head ((e >> 3) & 63): this
+      // thread's words belong to heads wt/8 (even steps) and wt/8 + 32 (odd)
       sm100::mbar_wait(&S.bar_q, 0, abort);
-      uint4* qv = reinterpret_cast<uint4*>(&S.q[0][0]);
+      const uint4* qv = reinterpret_cast<const uint4*>(&S.q[0][0]);
+      uint32_t ma = 0, mb = 0;
 #pragma unroll 4
-      for (int e = wt; e < 8 * kHg * 128 / 16; e += kThreads) qv[e] = bf16x8_to_f16(qv[e]);
+      for (int e = wt; e < 8 * kHg * 128 / 16; e += 2 * kThreads) {
+        ma = max(ma, bf16x8_amax_bits(qv[e]));
+        mb = max(mb, bf16x8_amax_bits(qv[e + kThreads]));
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, o));
+        mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+      }
+      if ((lane & 7) == 0) {
+        atomicMax(&S.qamax[wt >> 3], ma << 16);
+        atomicMax(&S.qamax[(wt >> 3) + 32], mb << 16);
+      }
     }
     // Conversion work: (8-row block, group of four 16-byte chunks) pairs,
     // one pair per warp instruction, lane = 4 x row-in-block + chunk-in-group:
     // both the staging reads and the swizzled V' stores then spread a warp's
     // 32 x 16 bytes over all banks.
     sm100::mbar_wait(&S.bar_g, i & 1, abort);
+    if (wt < kRows) {
+      // row prep: the row's largest RoPE magnitude, its shift k_j and the
+      // factors of its codes, RoPE dims, logits and denominator terms
+      const uint4* rp = reinterpret_cast<const uint4*>(stg + wt * kRowBytes + kNope);
+      uint32_t rb = 0;
+#pragma unroll
+      for (int x = 0; x < 2 * kR / 16; ++x) rb = max(rb, bf16x8_amax_bits(rp[x]));
+      const float sc = S.scale[wt];
+      const int kr = row_shift(sc, rb);
+      const float cj = ldexpf(sc, -kr);
+      const bool live = S.live[wt] != 0;
+      S.code_mul[wt] = kr >= -24 ? __uint_as_float((uint32_t)(127 + kr) << 23) : 0.f;
+      S.rope_mul[wt] = ldexpf(1.f / sc, kr);
+      S.row_f[wt] = live ? tau * kLog2e * cj : 0.f;
+      S.row_lc[wt] = log2f(cj);
+      S.row_ic[wt] = 1.f / cj;
+    }
     uint4 raw[kLoads];
 #pragma unroll
     for (int k = 0; k < kLoads; ++k) {
@@ -318,7 +404,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       const int r = 8 * (pr / 9) + (lane >> 2), c = 4 * (pr % 9) + (lane & 3);
       raw[k] = *reinterpret_cast<const uint4*>(stg + r * kRowBytes + c * 16);
     }
-    __syncthreads();  // staging area read by all; scales and live flags visible
+    __syncthreads();  // staging area read by all; row factors, live flags, query amax visible
+    if (i == 0) {
+      // each head's power-of-two range factor 2^e_h: Q'_h = Q_h 2^-e_h has
+      // its largest magnitude in [2^14, 2^15)
+      auto head_exp = [&](int h) {
+        const uint32_t a = S.qamax[h];
+        return a ? min(126, max(-126, (int)((a >> 23) & 0xFFu) - 127 - 14)) : 0;
+      };
+      if (wt < kHg) S.qg[wt] = __uint_as_float((uint32_t)(127 + head_exp(wt)) << 23);
+      const float qia = __uint_as_float((uint32_t)(127 - head_exp(wt >> 3)) << 23);
+      const float qib = __uint_as_float((uint32_t)(127 - head_exp((wt >> 3) + 32)) << 23);
+      uint4* qv = reinterpret_cast<uint4*>(&S.q[0][0]);
+#pragma unroll 4
+      for (int e = wt; e < 8 * kHg * 128 / 16; e += 2 * kThreads) {
+        qv[e] = bf16x8_scale_to_f16(qv[e], qia);
+        qv[e + kThreads] = bf16x8_scale_to_f16(qv[e + kThreads], qib);
+      }
+    }
     // -- convert + store V' (empty and dropped rows as zeros: the staging
     //    area holds stale bytes there)
 #pragma unroll
@@ -327,21 +430,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       const int r = 8 * (pr / 9) + (lane >> 2), c = 4 * (pr % 9) + (lane & 3);
       const bool live = S.live[r] != 0;
       if (c < kNope / 16) {
-        // dims 16c .. 16c+15 -> K-chunk (16c)/64, 16-byte slots 2(c%4), 2(c%4)+1
+        // dims 16c .. 16c+15 -> K-chunk (16c)/64, 16-byte slots 2(c%4), 2(c%4)+1;
+        // codes times 2^k (exact down to 2^-24)
         uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-        if (live) e4m3x16_to_f16(raw[k], lo, hi);
+        if (live) {
+          e4m3x16_to_f16(raw[k], lo, hi);
+          const float cm = S.code_mul[r];
+          if (cm != 1.f) {
+            const __half2 f = __float2half2_rn(cm);
+            __half2* ph = reinterpret_cast<__half2*>(&lo);
+            __half2* qh = reinterpret_cast<__half2*>(&hi);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) { ph[x] = __hmul2(ph[x], f); qh[x] = __hmul2(qh[x], f); }
+          }
+        }
         uint8_t* ch = S.v[c >> 2];
         *reinterpret_cast<uint4*>(ch + sw128(r, 2 * (c & 3))) = lo;
         *reinterpret_cast<uint4*>(ch + sw128(r, 2 * (c & 3) + 1)) = hi;
       } else {
-        // RoPE dims 448 + 8(c-28) .. : chunk 7, slot (c-28)
-        const uint4 v = live ? bf16x8_scale_to_f16(raw[k], S.inv_scale[r]) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(S.v[7] + sw128(r, c - kNope / 16)) = v;
+        // RoPE dims 448 + 8(c-28) .. times 2^k / s: hi in chunk 7 (slot
+        // c-28, read by both MMAs), lo at the same place of the P' buffer
+        // (free until the softmax; read by the S MMA only)
+        uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
+        if (live) bf16x8_scale_to_f16_hilo(raw[k], S.rope_mul[r], hi, lo);
+        *reinterpret_cast<uint4*>(S.v[7] + sw128(r, c - kNope / 16)) = hi;
+        *reinterpret_cast<uint4*>(S.p + sw128(r, c - kNope / 16)) = lo;
       }
     }
     sm100::fence_proxy_async_smem();
     __syncthreads();
-    // -- S^T = V' Q^T over K = 512 (32 steps of 16)
+    // -- S^T = V' Q^T over K = 512 (32 steps of 16), plus the RoPE dims'
+    //    lo parts against the query's RoPE dims (4 steps)
     if (issuer) {
       sm100::tc_fence_after();
       if (!*abort) {
@@ -351,6 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
           const uint32_t oq = (uint32_t)((kk >> 2) * kHg * 128 + (kk & 3) * 32);
           sm100::mma_f16(s_col, dadd(dV, o), dadd(dQ, oq), idS, kk > 0);
         }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          sm100::mma_f16(s_col, dadd(dPk, (uint32_t)(kk * 32)), dadd(dQ, (uint32_t)(7 * kHg * 128 + kk * 32)), idS, 1u);
         sm100::tc_commit(&S.bar_s);
       }
     }
@@ -359,15 +481,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     int64_t nx_off = -1;
     float nx_sc = 1.f;
     if (wt < kRows && i + 1 < n_tiles) {
-      nx_src = resolve_slot<kDense>(tb + kRows + wt, se, n_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap,
-                                    err, &nx_off);
+      nx_src = resolve_slot<kDense>(tb + kRows + wt, se, own_sel, t, n_t, W, bs, qi, idx, topk, cache_cap,
+                                    win_cap, err, &nx_off);
       if (nx_src) sm100::bulk_prefetch_l2((nx_src == 2 ? win_rows : cache_rows) + nx_off * kRowBytes, kRowBytes);
       if (nx_src == 1) nx_sc = cache_scale[nx_off];
       if (nx_src == 2) nx_sc = win_scale[nx_off];
     }
     sm100::mbar_wait(&S.bar_s, i & 1, abort);
     sm100::tc_fence_after();
-    // -- logits of this thread's row for its 32 heads
+    // -- this thread's row: c_j = s_j 2^-k_j, and u = z + log2 c_j (base-2
+    //    logit plus the row's log-scale) for its 32 heads
+    const float inv_c = S.row_ic[j];  // 1 / c_j
     float z[32];
     {
       uint32_t a[16], b[16];
@@ -376,12 +500,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       sm100::tmem_ld_x16(ta + 16, b);
       sm100::tmem_ld_wait();
       const bool valid = S.live[j] != 0;
-      const float f = tau * kLog2e * S.scale[j];
+      const float f = S.row_f[j];
+      const float lc = S.row_lc[j];
+      bool bad = false;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        z[c] = valid ? f * __uint_as_float(a[c]) : -INFINITY;
-        z[16 + c] = valid ? f * __uint_as_float(b[c]) : -INFINITY;
+        const float za = f * S.qg[32 * half + c] * __uint_as_float(a[c]);
+        const float zb = f * S.qg[32 * half + 16 + c] * __uint_as_float(b[c]);
+        const bool ba = !(fabsf(za) < INFINITY), bb = !(fabsf(zb) < INFINITY);
+        bad |= valid && (ba || bb);
+        z[c] = (valid && !ba) ? za + lc : -INFINITY;
+        z[16 + c] = (valid && !bb) ? zb + lc : -INFINITY;
       }
+      if (bad) raise_err(err, CSA_DEV_ERR_RANGE);  // a logit beyond fp32: dropped
     }
     // per-head tile maxima
     {
@@ -429,10 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       }
       sm100::tmem_st_wait();
     }
-    // probabilities, P' stores (row j, heads 32*half .. +31 = four 16-byte
-    // words) and per-head sums
+    // P' = exp2(u - m_h) (FP16 stores: row j, heads 32*half .. +31 = four
+    // 16-byte words) and the per-head sums of exp2(z - m_h) = P' / c_j
     {
-      const float sj = S.scale[j];
       float v[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
@@ -442,10 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
 #pragma unroll
       for (int w4 = 0; w4 < 4; ++w4) {
         const int b = 8 * w4;
-        const uint4 pk = make_uint4(pack_half2(v[b] * sj, v[b + 1] * sj), pack_half2(v[b + 2] * sj, v[b + 3] * sj),
-                                    pack_half2(v[b + 4] * sj, v[b + 5] * sj), pack_half2(v[b + 6] * sj, v[b + 7] * sj));
+        const uint4 pk = make_uint4(pack_half2(v[b], v[b + 1]), pack_half2(v[b + 2], v[b + 3]),
+                                    pack_half2(v[b + 4], v[b + 5]), pack_half2(v[b + 6], v[b + 7]));
         *reinterpret_cast<uint4*>(S.p + sw128(j, 4 * half + w4)) = pk;
       }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] *= inv_c;
       S.red[warp][lane] = warp_transpose_reduce32<false>(v);
     }
     sm100::tc_fence_before();
@@ -505,7 +637,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     float f[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) f[c] = S.alpha[32 * half + c];
-    uint16_t* stage = reinterpret_cast<uint16_t*>(&S.v[0][0]);  // [64 heads][512 dims]
+    // [64 heads][512 dims]: BF16 output, or the fp32 partial (128 KB, all of V')
+    uint16_t* stage = reinterpret_cast<uint16_t*>(&S.v[0][0]);
+    float* stage32 = reinterpret_cast<float*>(&S.v[0][0]);
 #pragma unroll 1
     for (int b2 = 0; b2 < 4; b2 += 2) {
       // four TMEM loads in flight: blocks b2, b2+1, this warp's 32 heads
@@ -530,25 +664,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
           const int hl = 16 * g + c;
           const int h = 32 * half + hl;
           float y = __uint_as_float(rr[x][c]) * f[hl];
-          uint16_t bits;
           if (single) {
             const float pv = __shfl_xor_sync(0xffffffffu, y, 1);
             if (c_dim >= kNope) y = odd ? (pv * sn + y * cs) : (y * cs - pv * sn);
-            bits = f32_to_bf16_bits(y);
+            stage[h * kD + c_dim] = f32_to_bf16_bits(y);
           } else {
-            bits = __half_as_ushort(__float2half_rn(y));
+            stage32[h * kD + c_dim] = y;
           }
-          stage[h * kD + c_dim] = bits;
         }
       }
     }
     __syncthreads();
-    // 64 rows of 1 KB, 16-byte words: row h = u / 64, word u % 64
-    uint16_t* dst0 = single ? out + ((int64_t)qi * n_heads + h0) * kD
-                            : reinterpret_cast<uint16_t*>(ws_o) + (((int64_t)qi * n_splits + split) * n_heads + h0) * kD;
+    // 64 rows of 1 KB (BF16) or 2 KB (fp32), 16-byte words
+    if (single) {
+      uint4* dst0 = reinterpret_cast<uint4*>(out + ((int64_t)qi * n_heads + h0) * kD);
 #pragma unroll 4
-    for (int u = wt; u < kHg * kD / 8; u += kThreads)
-      reinterpret_cast<uint4*>(dst0)[u] = reinterpret_cast<const uint4*>(stage)[u];
+      for (int u = wt; u < kHg * kD / 8; u += kThreads) dst0[u] = reinterpret_cast<const uint4*>(stage)[u];
+    } else {
+      uint4* dst0 = reinterpret_cast<uint4*>(ws_o + (((int64_t)qi * n_splits + split) * n_heads + h0) * kD);
+#pragma unroll 4
+      for (int u = wt; u < kHg * kD / 4; u += kThreads) dst0[u] = reinterpret_cast<const uint4*>(stage32)[u];
+    }
     if (!single && wt < kHg) {
       const int64_t base = ((int64_t)qi * n_splits + split) * n_heads + h0 + wt;
       ws_ml[base * 2 + 0] = S.mh[wt] * (1.0f / kLog2e);  // natural units
@@ -565,15 +701,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   }
 }
 
-// Combine the FP16 split partials (each O_s / l_s) of one query: for head h,
+// Combine the fp32 split partials (each O_s / l_s) of one query: for head h,
 // M = max(sink, m_s), w_s = l_s e^(m_s - M) / (e^(sink - M) + sum l_s
 // e^(m_s - M)), o = sum_s w_s (O_s / l_s) in split order, then the inverse
 // RoPE and a BF16 store.  grid (queries, n_heads / 8), 256 threads: warp =
 // head, lane = 16 dims.  The (m, l) of the first 32 splits are read once,
 // one split per lane, and shared by shuffles.
-__global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__ ws_o, const float* __restrict__ ws_ml,
+__global__ void __launch_bounds__(256) attn_merge_f32(const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
                                                       int n_splits, int n_heads, const float* __restrict__ sink,
-                                                      const int32_t* __restrict__ q_pos0, int T, float theta,
+                                                      const int32_t* __restrict__ q_pos0, int T, int m, int W,
+                                                      int n_sel, int dense, int rows_per_split, float theta,
                                                       uint16_t* __restrict__ out) {
   __shared__ float rope_c[kR / 2], rope_s[kR / 2];
   pdl_wait();
@@ -581,6 +718,11 @@ __global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__
   const int h = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int bs = qi / T, tq = qi % T;
   const int64_t t = (int64_t)q_pos0[bs] + tq;
+  // the query's own split count (a query with one split was finalised by
+  // attn_tc itself); n_splits is only the workspace stride
+  const int own_sel = dense ? (int)min((int64_t)n_sel, (t + 1) / m) : n_sel;
+  const int own_splits = (own_sel + W + rows_per_split - 1) / rows_per_split;
+  if (own_splits <= 1) return;
   if (threadIdx.x < kR / 2) {
     float c, sn;
     rope_cos_sin(-(double)t, threadIdx.x, kR, (double)theta, &c, &sn);
@@ -590,16 +732,16 @@ __global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__
   const float sg = sink[h];
   const int64_t ml0 = ((int64_t)qi * n_splits * n_heads + h) * 2;  // split sp at ml0 + 2 sp n_heads
   float m_l = -INFINITY, l_l = 0.f;
-  if (lane < n_splits) {
+  if (lane < own_splits) {
     m_l = ws_ml[ml0 + (int64_t)2 * lane * n_heads];
     l_l = ws_ml[ml0 + (int64_t)2 * lane * n_heads + 1];
   }
   float M = fmaxf(sg, warp_max(m_l));
-  for (int sp = 32 + lane; sp < n_splits; sp += 32) M = fmaxf(M, ws_ml[ml0 + (int64_t)2 * sp * n_heads]);
+  for (int sp = 32 + lane; sp < own_splits; sp += 32) M = fmaxf(M, ws_ml[ml0 + (int64_t)2 * sp * n_heads]);
   M = warp_max(M);
   const float p_l = (m_l == -INFINITY) ? 0.f : l_l * expf(m_l - M);  // split `lane`
   float part = p_l;
-  for (int sp = 32 + lane; sp < n_splits; sp += 32) {
+  for (int sp = 32 + lane; sp < own_splits; sp += 32) {
     const float ms = ws_ml[ml0 + (int64_t)2 * sp * n_heads];
     if (ms != -INFINITY) part += ws_ml[ml0 + (int64_t)2 * sp * n_heads + 1] * expf(ms - M);
   }
@@ -610,9 +752,9 @@ __global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-  const __half* src0 = ws_o + ((int64_t)qi * n_splits * n_heads + h) * kD + c0;
+  const float* src0 = ws_o + ((int64_t)qi * n_splits * n_heads + h) * kD + c0;
 #pragma unroll 4
-  for (int sp = 0; sp < n_splits; ++sp) {
+  for (int sp = 0; sp < own_splits; ++sp) {
     float a;
     if (sp < 32) {
       a = __shfl_sync(0xffffffffu, a_l, sp);
@@ -621,17 +763,14 @@ __global__ void __launch_bounds__(256) attn_merge_f16(const __half* __restrict__
       a = ms == -INFINITY ? 0.f : ws_ml[ml0 + (int64_t)2 * sp * n_heads + 1] * expf(ms - M) * inv;
     }
     if (a == 0.f) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(src0 + (int64_t)sp * n_heads * kD);
-    const uint4 v0 = src[0], v1 = src[1];
-    const __half2* p0 = reinterpret_cast<const __half2*>(&v0);
-    const __half2* p1 = reinterpret_cast<const __half2*>(&v1);
+    const float4* src = reinterpret_cast<const float4*>(src0 + (int64_t)sp * n_heads * kD);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f0 = __half22float2(p0[e]), f1 = __half22float2(p1[e]);
-      acc[2 * e] = fmaf(a, f0.x, acc[2 * e]);
-      acc[2 * e + 1] = fmaf(a, f0.y, acc[2 * e + 1]);
-      acc[8 + 2 * e] = fmaf(a, f1.x, acc[8 + 2 * e]);
-      acc[8 + 2 * e + 1] = fmaf(a, f1.y, acc[8 + 2 * e + 1]);
+      const float4 v = src[e];
+      acc[4 * e] = fmaf(a, v.x, acc[4 * e]);
+      acc[4 * e + 1] = fmaf(a, v.y, acc[4 * e + 1]);
+      acc[4 * e + 2] = fmaf(a, v.z, acc[4 * e + 2]);
+      acc[4 * e + 3] = fmaf(a, v.w, acc[4 * e + 3]);
     }
   }
   __syncthreads();  // rope table
@@ -677,31 +816,21 @@ bool attn_tc_supported(const csa_params& p) {
          p.n_heads % kHg == 0 && encode_fn() != nullptr;
 }
 
-// Rows per split.  Prefill (T > 4): all of a query's slots in one split.
-// Decode: t tiles per split, t minimising  waves x (c + t) + 0.05 x splits,
-// where waves = ceil(CTAs / SMs) (one CTA per SM), c = 0.7 tiles is the
-// fixed cost of a CTA (setup, query load, epilogue) and the last term the
-// merge's share per split.
-int attn_tc_rows_per_split(int total_slots, int nq, int nhg, int T) {
+// Rows per split, a function of the call's parameters and T only -- never
+// of the batch size, the other sequences' lengths or the device -- so that
+// a query's output is bit-identical whatever batch it runs in (the
+// batch-invariant contract of the DeepSeek-V4 write-ups: kwkr.cn notes 4.3,
+// Qiaomu blog 批次不变和确定性内核).  Prefill (T > 4): all of a query's slots
+// in one split.  Sparse decode (k + W slots, fixed by the parameters): up
+// to 16 tiles, splits of 2 tiles (one 64-head group) or 1 tile (several
+// groups already multiply the CTAs), else 8 tiles.  Dense decode (a query's
+// slot count is its own n_t + W): splits of 8 tiles.
+int attn_tc_rows_per_split(int total_slots, int nhg, int T, bool dense) {
   const int tiles = (total_slots + kRows - 1) / kRows;
-  if (T > 4 || tiles <= 1) return (tiles > 1 ? tiles : 1) * kRows;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (sms <= 0) sms = 148;
-  int best_t = 1;
-  double best = 1e300;
-  for (int t = 1; t <= tiles; ++t) {
-    const int64_t splits = (tiles + t - 1) / t;
-    const int64_t ctas = (int64_t)nq * nhg * splits;
-    const int64_t waves = (ctas + sms - 1) / sms;
-    const double cost = (double)waves * (0.7 + t) + 0.05 * (double)splits;
-    if (cost < best - 1e-9) {
-      best = cost;
-      best_t = t;
-    }
-  }
-  return best_t * kRows;
+  if (T > 4) return (tiles > 1 ? tiles : 1) * kRows;
+  if (dense) return 8 * kRows;
+  if (tiles <= 16) return (nhg == 1 ? 2 : 1) * kRows;
+  return 8 * kRows;
 }
 
 size_t attn_tc_smem_bytes() { return sizeof(AttnSmem) + 1024; }
@@ -723,13 +852,12 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
   }
   const int total = n_sel + p.window;
   const int nhg = p.n_heads / kHg;
-  const int rps = attn_tc_rows_per_split(total, nq, nhg, T);
+  const int rps = attn_tc_rows_per_split(total, nhg, T, dense);
   const int n_splits = (total + rps - 1) / rps;
-  // workspace: FP16 partials O/l, then (max, sum) per (query, split, head)
+  // workspace: fp32 partials O/l, then (max, sum) per (query, split, head)
   const size_t n_part = (size_t)nq * n_splits * p.n_heads;
-  __half* ws_o = reinterpret_cast<__half*>(ws);
-  float* ws_ml = ws ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ((n_part * p.d * 2 + 15) & ~(size_t)15))
-                    : nullptr;
+  float* ws_o = ws;
+  float* ws_ml = ws ? ws + n_part * p.d : nullptr;
   const size_t smem = attn_tc_smem_bytes();
   auto kfn = dense ? attn_tc<true> : attn_tc<false>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -740,18 +868,18 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
                  p.m, p.window, n_sel, p.n_heads, p.softmax_scale, p.rope_theta, sink, rps, n_splits,
                  reinterpret_cast<uint16_t*>(out), ws_o, ws_ml, err);
   if (e != cudaSuccess || n_splits == 1) return e;
-  return launch_pdl(attn_merge_f16, dim3(nq, p.n_heads / 8), dim3(256), 0, st, (const __half*)ws_o,
-                    (const float*)ws_ml, n_splits, p.n_heads, sink, q_pos0, T, p.rope_theta,
-                    reinterpret_cast<uint16_t*>(out));
+  return launch_pdl(attn_merge_f32, dim3(nq, p.n_heads / 8), dim3(256), 0, st, (const float*)ws_o,
+                    (const float*)ws_ml, n_splits, p.n_heads, sink, q_pos0, T, p.m, p.window, n_sel, dense ? 1 : 0,
+                    rps, p.rope_theta, reinterpret_cast<uint16_t*>(out));
 }
 
 size_t attn_tc_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense) {
   const int total = n_sel + p.window;
-  const int rps = attn_tc_rows_per_split(total, p.B * T, p.n_heads / kHg, T);
+  const int rps = attn_tc_rows_per_split(total, p.n_heads / kHg, T, dense);
   const int n_splits = (total + rps - 1) / rps;
   if (n_splits == 1) return 0;
   const size_t n_part = (size_t)p.B * T * n_splits * p.n_heads;
-  return ((n_part * p.d * 2 + 15) & ~(size_t)15) + n_part * 2 * sizeof(float);
+  return n_part * (p.d + 2) * sizeof(float);
 }
 
 }  // namespace csa

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -110,6 +111,44 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool acti
   const unsigned peers = __match_any_sync(act, bin);
   const int leader = __ffs(peers) - 1;
   if ((int)(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
+// Four consecutive values from f32 or BF16 storage (element offset `off`,
+// a multiple of 4).
+template <bool kF32>
+__device__ __forceinline__ void load4(const void* base, int64_t off, float v[4]) {
+  if (kF32) {
+    float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    uint2 x = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + off);
+    v[0] = bf16_bits_to_f32(x.x); v[1] = bf16_bits_to_f32(x.x >> 16);
+    v[2] = bf16_bits_to_f32(x.y); v[3] = bf16_bits_to_f32(x.y >> 16);
+  }
+}
+
+// OCP MX v1.0 conversion (section 6.3) of one 32-value block held as 4
+// values by each of 8 consecutive lanes (`mask` = those lanes): the shared
+// exponent is X = floor(log2 amax) - 2 (E2M1's largest exponent is 2),
+// clamped to [-127, 127] (an all-zero block takes -127), and each value
+// becomes the E2M1 code of v * 2^-X, rounded to nearest even and
+// saturated.  Returns this lane's two packed bytes (value 0 in the low
+// nibble of the low byte) and sets *sbyte = X + 127 (the UE8M0 scale).
+__device__ __forceinline__ uint32_t mxfp4_encode_quad(const float v[4], unsigned mask, uint32_t* sbyte) {
+  float am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  am = fmaxf(am, __shfl_xor_sync(mask, am, 1));
+  am = fmaxf(am, __shfl_xor_sync(mask, am, 2));
+  am = fmaxf(am, __shfl_xor_sync(mask, am, 4));
+  // floor(log2 am) from the exponent field; a subnormal (or zero) amax
+  // gives an exponent below -127 after the -2, i.e. the clamp
+  const int e = (int)((__float_as_uint(am) >> 23) & 0xFFu);
+  int X = e ? e - 127 - 2 : -127;
+  X = max(-127, min(125, X));
+  const float inv = __uint_as_float((uint32_t)(127 - X) << 23);  // 2^-X, X in [-127, 125]
+  const uint32_t b0 = __nv_cvt_float2_to_fp4x2(make_float2(v[0] * inv, v[1] * inv), __NV_E2M1, cudaRoundNearest);
+  const uint32_t b1 = __nv_cvt_float2_to_fp4x2(make_float2(v[2] * inv, v[3] * inv), __NV_E2M1, cudaRoundNearest);
+  *sbyte = (uint32_t)(X + 127);
+  return (b0 & 0xFFu) | ((b1 & 0xFFu) << 8);
 }
 
 // Bins of the per-query score histogram: the top 12 bits of the key.

@@ -15,19 +15,11 @@
 
 namespace csa {
 
-template <bool kF32>
-__device__ __forceinline__ void load4(const void* base, int64_t off, float v[4]) {
-  if (kF32) {
-    float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
-    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-  } else {
-    uint2 x = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + off);
-    v[0] = bf16_bits_to_f32(x.x); v[1] = bf16_bits_to_f32(x.x >> 16);
-    v[2] = bf16_bits_to_f32(x.y); v[3] = bf16_bits_to_f32(x.y >> 16);
-  }
-}
+// Output of the compressor: f32 rows, the mixed FP8/BF16 KV rows, or MXFP4
+// index-key rows (the indexer's keys come from the same operator).
+enum { kOutF32 = 0, kOutFp8 = 1, kOutMxfp4 = 2 };
 
-template <bool kF32, bool kKvF32>
+template <bool kF32, int kOut>
 __global__ void __launch_bounds__(1024) compress_kernel(
     const csa_params p, const void* __restrict__ a, const void* __restrict__ b,
     const float* __restrict__ gate, int64_t S, const int32_t* __restrict__ tok_base,
@@ -151,7 +143,17 @@ __global__ void __launch_bounds__(1024) compress_kernel(
   }
   const int64_t slot = (int64_t)bs * cap + e;
   if (out_pos && threadIdx.x == 0) out_pos[slot] = (int32_t)(m * e);
-  if (kKvF32) {
+  if (kOut == kOutMxfp4) {
+    // OCP MX conversion per 32 dims: eight consecutive owner lanes hold a
+    // block; 2 packed bytes per lane, one scale byte per block
+    const unsigned mask = 0xFFu << (threadIdx.x & 24);
+    uint32_t sb;
+    const uint32_t bytes = mxfp4_encode_quad(y, mask, &sb);
+    reinterpret_cast<uint16_t*>(rows + slot * (d / 2))[q] = (uint16_t)bytes;
+    if ((q & 7) == 0) reinterpret_cast<uint8_t*>(scale)[slot * (d / 32) + (q >> 3)] = (uint8_t)sb;
+    return;
+  }
+  if (kOut == kOutF32) {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(rows) + slot * d + d0) =
         make_float4(y[0], y[1], y[2], y[3]);
     return;
@@ -197,10 +199,62 @@ cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, c
   dim3 grid(max_entries, p.B);
   const bool f32 = p.act_fmt == CSA_ACT_F32, kv32 = p.kv_fmt == CSA_KV_F32;
   auto* rows = reinterpret_cast<uint8_t*>(out.rows);
-  auto kfn = f32 ? (kv32 ? compress_kernel<true, true> : compress_kernel<true, false>)
-                 : (kv32 ? compress_kernel<false, true> : compress_kernel<false, false>);
+  auto kfn = f32 ? (kv32 ? compress_kernel<true, kOutF32> : compress_kernel<true, kOutFp8>)
+                 : (kv32 ? compress_kernel<false, kOutF32> : compress_kernel<false, kOutFp8>);
   cudaError_t e = launch_pdl(kfn, grid, dim3(threads), smem, st, p, a, b, gate, S, tok_base, e_begin, e_end, norm_w,
                              rows, out.scale, out.cap, out_pos, err);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Index keys: the compressor over the idx_dim-dim indexer streams with RoPE
+// on their last rope_dims dims, written as MXFP4 rows (idx_dim/2 bytes) and
+// UE8M0 scales (idx_dim/32 bytes) per entry.
+cudaError_t launch_index_compress(const csa_params& p, int rope_dims, const void* a, const void* b,
+                                  const float* gate, int64_t S, const int32_t* tok_base, const int32_t* e_begin,
+                                  const int32_t* e_end, int32_t max_entries, const float* norm_w, void* k_idx,
+                                  uint8_t* k_idx_sf, int64_t k_cap, int32_t* err, cudaStream_t st) {
+  csa_params q = p;
+  q.d = p.idx_dim;
+  q.r = rope_dims;
+  const int quads = q.d / 4;
+  const int threads = 256;
+  const int G = threads / quads;
+  const size_t smem = (size_t)(2 * q.m + G * q.d) * sizeof(float);
+  dim3 grid(max_entries, p.B);
+  auto kfn = p.act_fmt == CSA_ACT_F32 ? compress_kernel<true, kOutMxfp4> : compress_kernel<false, kOutMxfp4>;
+  cudaError_t e = launch_pdl(kfn, grid, dim3(threads), smem, st, q, a, b, gate, S, tok_base, e_begin, e_end, norm_w,
+                             reinterpret_cast<uint8_t*>(k_idx), reinterpret_cast<float*>(k_idx_sf), k_cap,
+                             (int32_t*)nullptr, err);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Index queries (or any rows of idx_dim values) to MXFP4 by the OCP MX
+// conversion: one thread per 4 values, eight threads per 32-value block.
+template <bool kF32>
+__global__ void __launch_bounds__(256) index_quantize_kernel(const void* __restrict__ x, int64_t n_quads,
+                                                             uint8_t* __restrict__ out, uint8_t* __restrict__ out_sf) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g - (threadIdx.x & 7) >= n_quads) return;  // whole 8-lane groups leave together
+  float v[4];
+  load4<kF32>(x, g * 4, v);
+  uint32_t sb;
+  const uint32_t bytes = mxfp4_encode_quad(v, 0xFFu << (threadIdx.x & 24), &sb);
+  reinterpret_cast<uint16_t*>(out)[g] = (uint16_t)bytes;
+  if ((threadIdx.x & 7) == 0) out_sf[g >> 3] = (uint8_t)sb;
+}
+
+cudaError_t launch_index_quantize(const csa_params& p, const void* x, int64_t n_rows, void* out, uint8_t* out_sf,
+                                  cudaStream_t st) {
+  const int64_t n_quads = n_rows * (p.idx_dim / 4);
+  if (n_quads == 0) return cudaSuccess;
+  const int64_t blocks = (n_quads + 255) / 256;
+  auto kfn = p.act_fmt == CSA_ACT_F32 ? index_quantize_kernel<true> : index_quantize_kernel<false>;
+  cudaError_t e = launch_pdl(kfn, dim3((unsigned)blocks), dim3(256), 0, st, x, n_quads, reinterpret_cast<uint8_t*>(out),
+                             out_sf);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

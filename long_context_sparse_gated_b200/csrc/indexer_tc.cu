@@ -8,26 +8,33 @@
 //                                            B = the query's 64 heads)
 //   I(t, s) = sum_h w_h * max(D[s, h], 0)   (epilogue, fp32, h = 0..63)
 //
-// Persistent, warp-specialised CTA (one per SM), 320 threads:
-//   warp 0     TMA producer: per tile the 128x64 B key block (64B swizzle,
-//              rows permuted by a 3-D view, see Stage) and its 512 scale
-//              bytes into a kStages-deep ring; per query (not per tile) the
-//              64x64 B query block and its scales into one of two slots
+// Persistent, warp-specialised CTA (one per SM), 320 threads, walking
+// stages of 256 entries (two 128-entry MMA tiles):
+//   warp 0     TMA producer: per stage two 128x64 B key boxes (64B swizzle,
+//              rows permuted by a 3-D view, see Stage) and the stage's 1 KB
+//              of scales into a kStages-deep ring; per query (not per
+//              stage) the 64x64 B query block and its scales into one of
+//              two slots
 //   warp 1     MMA issuer (one lane): per query, permutes the query scales
-//              into the 32x16 B layout and copies them to TMEM; per tile,
-//              copies the key scales to TMEM (tcgen05.cp), issues two K=64
-//              MMAs into one of four TMEM accumulators and commits them
-//   warps 2-9  two epilogue warpgroups taking alternate tiles: once a
-//              tile's MMAs are complete they release its shared-memory stage
-//              to the producer, tcgen05.ld the 64 head columns of one entry
-//              per thread, ReLU, weighted head sum (four independent partial
-//              sums), fp32 store, and (optionally) count the score's top 12
-//              key bits into the warpgroup's shared-memory histogram of the
-//              current query, which is added to the global per-query
-//              histogram (the top-k selector's starting point) when the
-//              warpgroup moves to another query and at the end
-// Each CTA walks a contiguous range of (query, 128-entry block) tiles, so the
-// key stream it reads is sequential.  Tiles past a query's n_t are skipped.
+//              into the 32x16 B layout and copies them to TMEM; per stage,
+//              copies the two tiles' key scales to TMEM (tcgen05.cp), issues
+//              four K=64 MMAs (two per tile) into one of three TMEM
+//              accumulator pairs, and commits twice: to the pair's "full"
+//              barrier and to the stage's "empty" barrier, so the ring slot
+//              goes back to the producer as soon as the MMAs have read it
+//   warps 2-9  two epilogue warpgroups; warpgroup g takes tile g of every
+//              stage: once the stage's MMAs are complete it tcgen05.ld's the
+//              64 head columns of one entry per thread, frees the
+//              accumulator, applies ReLU and the weighted head sum (four
+//              independent partial sums), stores the fp32 score and
+//              (optionally) counts the score's top 12 key bits into the
+//              warpgroup's shared-memory histogram of the current query,
+//              which is added to the global per-query histogram (the top-k
+//              selector's starting point) when the warpgroup moves to
+//              another query and at the end
+// Each CTA walks a contiguous range of (query, 256-entry block) stages, so
+// the key stream it reads is sequential.  Stages past a query's n_t are
+// skipped.
 //
 // Numerics: with MXFP4 inputs whose per-32 scales are >= 2^-2 and dyadic
 // head weights, every partial sum is exactly representable in fp32 (the
@@ -42,15 +49,17 @@ namespace csa {
 
 namespace {
 
-constexpr int kStages = 12;
-constexpr int kTileM = 128;   // entries per tile
+constexpr int kStages = 10;
+constexpr int kTileM = 128;   // entries per MMA tile
+constexpr int kTiles = 2;     // MMA tiles per stage
+constexpr int kStageKeys = kTileM * kTiles;     // 256 entries per stage
 constexpr int kHeads = 64;    // index heads (N)
 constexpr int kRowBytes = 64; // 128 E2M1 values
-constexpr int kKeyBytes = kTileM * kRowBytes;   // 8192
+constexpr int kKeyBytes = kTileM * kRowBytes;   // 8192 per tile
 constexpr int kQBytes = kHeads * kRowBytes;     // 4096
-constexpr int kSfkBytes = kTileM * 4;           // 512 (4 UE8M0 per row)
+constexpr int kSfkBytes = kTileM * 4;           // 512 per tile (4 UE8M0 per row)
 constexpr int kSfqBytes = kHeads * 4;           // 256
-constexpr uint32_t kStageTx = kKeyBytes + kSfkBytes;
+constexpr uint32_t kStageTx = kTiles * (kKeyBytes + kSfkBytes);
 constexpr uint32_t kQueryTx = kQBytes + kSfqBytes;
 
 // A tile's 128 keys are loaded through a 3-D view of the key array, so that
@@ -59,8 +68,8 @@ constexpr uint32_t kQueryTx = kQBytes + kSfqBytes;
 // tcgen05.cp expects (line i = scale words of MMA rows i, 32+i, 64+i, 96+i),
 // and no per-tile permutation is needed.
 struct __align__(1024) Stage {
-  uint8_t key[kKeyBytes];   // 1024-aligned (64B-swizzle atoms are 512 B)
-  uint32_t sfk[kTileM];
+  uint8_t key[kTiles][kKeyBytes];   // 1024-aligned (64B-swizzle atoms are 512 B)
+  uint32_t sfk[kTiles][kTileM];     // the stage's 256 scale words, in entry order
 };
 
 struct __align__(1024) QuerySlot {
@@ -69,8 +78,8 @@ struct __align__(1024) QuerySlot {
   uint32_t sfq[kTileM];     // permuted for tcgen05.cp; rows 64..127 zero
 };
 
-constexpr int kAcc = 4;         // TMEM accumulators (two per epilogue warpgroup)
-constexpr int kEpiGroups = 2;   // epilogue warpgroups, alternating tiles
+constexpr int kAcc = 3;         // TMEM accumulator pairs (one tile each per epilogue warpgroup)
+constexpr int kEpiGroups = kTiles;  // epilogue warpgroup g takes tile g of every stage
 constexpr int kHistBins = 4096; // score histogram bins (top 12 key bits)
 
 struct Smem {
@@ -87,11 +96,11 @@ struct Smem {
   int abort;
 };
 
-// TMEM columns: accumulators 0..255, key scales 256 + 4 acc, query scales
-// 272 + 4 slot.
+// TMEM columns: accumulator pair a, tile g at 128 a + 64 g (0..383); key
+// scales 384 + 8 a + 4 g; query scales 408 + 4 slot.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfaCol = kAcc * kHeads;
-constexpr uint32_t kSfbCol = kSfaCol + 4 * kAcc;
+constexpr uint32_t kSfaCol = kAcc * kTiles * kHeads;
+constexpr uint32_t kSfbCol = kSfaCol + 4 * kTiles * kAcc;
 
 __device__ __forceinline__ int visible(const int32_t* q_pos0, int T, int m, int qi, int n_max) {
   const int bs = qi / T, tq = qi % T;
@@ -142,7 +151,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tpq = (n_max + kTileM - 1) / kTileM;  // tiles per query
+  const int tpq = (n_max + kStageKeys - 1) / kStageKeys;  // stages per query
   const int64_t n_tiles = (int64_t)n_queries * tpq;
   const int64_t t_begin = n_tiles * blockIdx.x / gridDim.x;
   const int64_t t_end = n_tiles * (blockIdx.x + 1) / gridDim.x;
@@ -159,7 +168,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     }
     for (int i = 0; i < kAcc; ++i) {
       sm100::mbar_init(&S.tfull[i], 1);
-      sm100::mbar_init(&S.tempty[i], 4);
+      sm100::mbar_init(&S.tempty[i], 4 * kEpiGroups);
     }
     S.abort = 0;
     sm100::fence_mbar_init();
@@ -187,7 +196,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       int bs = 0;
       for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
         const int qi = c.qi, j = c.j;
-        if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
+        if (j * kStageKeys >= vc.get(q_pos0, T, m, qi, n_max)) continue;
         if (qi != cur_q) {  // the query's 64 heads, once per query
           bs = qi / T;
           const int sl = nq & 1;
@@ -203,8 +212,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         if (!sm100::mbar_wait(&S.empty[s], ph ^ 1, abort)) break;
         Stage& st = S.st[s];
         sm100::mbar_arrive_expect_tx(&S.full[s], kStageTx);
-        const int64_t row = (int64_t)bs * k_cap + (int64_t)j * kTileM;
-        sm100::tma_load_3d(st.key, &tm_key, &S.full[s], 0, (int32_t)(row / 4), 0);
+        const int64_t row = (int64_t)bs * k_cap + (int64_t)j * kStageKeys;
+        sm100::tma_load_3d(st.key[0], &tm_key, &S.full[s], 0, (int32_t)(row / 4), 0);
+        sm100::tma_load_3d(st.key[1], &tm_key, &S.full[s], 0, (int32_t)(row / 4) + kTileM / 4, 0);
         sm100::tma_load_1d(st.sfk, &tm_sfk, &S.full[s], (int32_t)row);
         ++it;
       }
@@ -217,7 +227,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       VisibleCache vc;
       for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
         const int qi = c.qi, j = c.j;
-        if (j * kTileM >= vc.get(q_pos0, T, m, qi, n_max)) continue;
+        if (j * kStageKeys >= vc.get(q_pos0, T, m, qi, n_max)) continue;
         if (qi != cur_q) {
           // the previous query's slot is free once its MMAs complete
           if (cur_q >= 0) sm100::tc_commit(&S.qempty[sl]);
@@ -241,28 +251,33 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         if (!sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort) || !sm100::mbar_wait(&S.full[s], ph, abort)) break;
         sm100::tc_fence_after();
         Stage& st = S.st[s];
-        const uint32_t d_col = tmem + acc * kHeads;
-        const uint32_t sfa_col = tmem + kSfaCol + 4 * acc;
         const uint32_t sfb_col = tmem + kSfbCol + 4 * sl;
-        sm100::tc_cp_32x128b_warpx4(sfa_col, sm100::smem_desc(sm100::smem_u32(st.sfk), 0, 128, 0));
-        const uint32_t ka = sm100::smem_u32(st.key), qa = sm100::smem_u32(S.qs[sl].q);
+        const uint32_t qa = sm100::smem_u32(S.qs[sl].q);
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          // K elements [64kk, 64kk+64) = bytes [32kk, 32kk+32) of every row
-          const uint64_t adesc = sm100::smem_desc(ka + 32 * kk, 16, 512, 4);
-          const uint64_t bdesc = sm100::smem_desc(qa + 32 * kk, 16, 512, 4);
-          sm100::mma_mxf4(d_col, adesc, bdesc, sm100::idesc_mxf4(kTileM, kHeads, 2 * kk, 2 * kk), sfa_col,
-                          sfb_col, kk);
+        for (int g = 0; g < kTiles; ++g) {
+          const uint32_t d_col = tmem + (acc * kTiles + g) * kHeads;
+          const uint32_t sfa_col = tmem + kSfaCol + 4 * (acc * kTiles + g);
+          sm100::tc_cp_32x128b_warpx4(sfa_col, sm100::smem_desc(sm100::smem_u32(st.sfk[g]), 0, 128, 0));
+          const uint32_t ka = sm100::smem_u32(st.key[g]);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            // K elements [64kk, 64kk+64) = bytes [32kk, 32kk+32) of every row
+            const uint64_t adesc = sm100::smem_desc(ka + 32 * kk, 16, 512, 4);
+            const uint64_t bdesc = sm100::smem_desc(qa + 32 * kk, 16, 512, 4);
+            sm100::mma_mxf4(d_col, adesc, bdesc, sm100::idesc_mxf4(kTileM, kHeads, 2 * kk, 2 * kk), sfa_col,
+                            sfb_col, kk);
+          }
         }
-        // completion frees the accumulator's inputs: the epilogue releases
-        // the stage to the producer once it has seen this commit
+        // completion: the accumulator pair is ready for the epilogue, and
+        // the stage's shared memory goes back to the producer
         sm100::tc_commit(&S.tfull[acc]);
+        sm100::tc_commit(&S.empty[s]);
         ++it;
       }
     }
   } else {
     // ---------------- epilogue (warps 2..9: two warpgroups) ----------------
-    const int eg = (warp - 2) >> 2;  // warpgroup: tiles it with it % 2 == eg
+    const int eg = (warp - 2) >> 2;  // warpgroup: tile eg of every stage
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     // TMEM lane 32*quad + lane holds key 4*lane + quad of the tile
     const int key_in_tile = 4 * lane + quad;
@@ -291,9 +306,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
       const int qi = c.qi, j = c.j;
       const int n_t = vc.get(q_pos0, T, m, qi, n_max);
-      if (j * kTileM >= n_t) continue;
+      if (j * kStageKeys >= n_t) continue;
       const uint32_t my = it++;
-      if ((int)(my % kEpiGroups) != eg) continue;
       const int acc = my % kAcc;
       const uint32_t aph = (my / kAcc) & 1;
       if (qi != wq) {  // head weights of this tile's query, kept in registers
@@ -307,18 +321,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         wq = qi;
       }
       int ok = 1;
-      if (lane == 0) {
-        ok = sm100::mbar_wait(&S.tfull[acc], aph, abort);
-        // the tile's MMAs are complete: its key stage may be refilled
-        if (ok && quad == 0) sm100::mbar_arrive(&S.empty[my % kStages]);
-      }
+      if (lane == 0) ok = sm100::mbar_wait(&S.tfull[acc], aph, abort);
       // no break on a failed wait: every warp of the warpgroup keeps walking
       // the same tiles so that the histogram flushes' named barriers match;
       // after an abort every wait returns at once and no work is done
       if (!__shfl_sync(0xffffffffu, ok, 0)) continue;
       sm100::tc_fence_after();
       uint32_t d[64];
-      const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + acc * kHeads;
+      const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + (acc * kTiles + eg) * kHeads;
       sm100::tmem_ld_x16(base + 0, *reinterpret_cast<uint32_t(*)[16]>(d + 0));
       sm100::tmem_ld_x16(base + 16, *reinterpret_cast<uint32_t(*)[16]>(d + 16));
       sm100::tmem_ld_x16(base + 32, *reinterpret_cast<uint32_t(*)[16]>(d + 32));
@@ -333,7 +343,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
 #pragma unroll
       for (int h = 0; h < kHeads; ++h) p4[h & 3] = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), p4[h & 3]);
       const float sc = (p4[0] + p4[1]) + (p4[2] + p4[3]);
-      const int s_idx = j * kTileM + key_in_tile;
+      const int s_idx = j * kStageKeys + eg * kTileM + key_in_tile;
       if (s_idx < n_t) {
         scores[(int64_t)qi * ld + s_idx] = sc;
         if (hist) atomicAdd(sh + score_bin(sc), 1u);
@@ -416,7 +426,7 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
   {
     uint64_t dims[1] = {key_rows};
     uint64_t str[1] = {4};
-    uint32_t box[1] = {kTileM};
+    uint32_t box[1] = {kStageKeys};
     if (!make_map(&tsk, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, k_sf, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
@@ -430,7 +440,7 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int tpq = (n_max + kTileM - 1) / kTileM;
+  const int tpq = (n_max + kStageKeys - 1) / kStageKeys;
   const int64_t tiles = (int64_t)nq * tpq;
   const int grid = (int)(tiles < sms ? tiles : sms);
   if (grid == 0) return cudaSuccess;

@@ -9,6 +9,10 @@
 
 namespace csa {
 
+// Message returned by csa_last_error_string() on this host thread (a string
+// with static storage duration).
+void set_last_error(const char* msg);
+
 // Launch with programmatic stream serialisation (see pdl_wait in
 // common.cuh): the kernel may begin while its predecessor on the stream
 // drains.
@@ -32,6 +36,14 @@ cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, c
                             int64_t S, const int32_t* tok_base, const int32_t* e_begin,
                             const int32_t* e_end, int32_t max_entries, const float* norm_w,
                             const csa_kv& out, int32_t* out_pos, int32_t* err, cudaStream_t st);
+
+cudaError_t launch_index_compress(const csa_params& p, int rope_dims, const void* a, const void* b,
+                                  const float* gate, int64_t S, const int32_t* tok_base, const int32_t* e_begin,
+                                  const int32_t* e_end, int32_t max_entries, const float* norm_w, void* k_idx,
+                                  uint8_t* k_idx_sf, int64_t k_cap, int32_t* err, cudaStream_t st);
+
+cudaError_t launch_index_quantize(const csa_params& p, const void* x, int64_t n_rows, void* out, uint8_t* out_sf,
+                                  cudaStream_t st);
 
 cudaError_t launch_index_scores(const csa_params& p, const void* q_idx, const uint8_t* q_sf,
                                 const float* w, const void* k_idx, const uint8_t* k_sf,
@@ -57,7 +69,8 @@ cudaError_t launch_topk_select(const csa_params& p, const float* scores, int ld,
 size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense);
 
 cudaError_t launch_attn_merge(const csa_params& p, const float* ws_o, const float* ws_ml, int n_splits,
-                              const float* sink, const int32_t* q_pos0, int T, void* out, cudaStream_t st);
+                              const float* sink, const int32_t* q_pos0, int T, int n_sel, bool dense,
+                              int rows_per_split, void* out, cudaStream_t st);
 
 bool attn_tc_supported(const csa_params& p);
 size_t attn_tc_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense);

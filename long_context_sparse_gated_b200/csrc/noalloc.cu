@@ -10,19 +10,25 @@
 // file-scope static device array instead, so the caller passes only inputs
 // and outputs.
 //
-// The array holds kScratchBytes (16 MiB) on every GPU that loads the
-// library, from module load until the process exits.  Problems whose
-// workspace (csa_index_topk_workspace_bytes) exceeds it are rejected with
+// The array holds kScratchBytes (16 MiB).  It belongs to this file's module,
+// which the CUDA runtime loads on a device lazily: the first call on a device
+// loads it there (reserving the 16 MiB) and looks up the array's address;
+// the reservation then lasts until the process exits (or the device's
+// context is destroyed, after which the next call loads the module and looks
+// the address up again).  Problems whose workspace
+// (csa_index_topk_workspace_bytes) exceeds it are rejected with
 // CSA_ERR_WORKSPACE before anything is launched.  All calls share the one
 // array: two calls whose work overlaps on the GPU (different streams, or
 // different host threads on the same device) race on it; the array keeps the
 // previous call's contents, and the parts that must start at zero (the
 // histograms) are cleared on every call by the regular path.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "csa.h"
+#include "kernels.h"
 
 namespace {
 
@@ -33,21 +39,69 @@ constexpr int kMaxDevices = 64;
 // for the symbol; its device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_index_scratch[kScratchBytes];
 
-// Device address of g_index_scratch per device ordinal, looked up once per
-// device with that device current.
-void* g_scratch_addr[kMaxDevices] = {};
+// Device address of g_index_scratch per device ordinal, looked up with that
+// device current, together with the id of the context it belongs to (a
+// destroyed and re-created context gets a new id and a new address).
+struct ScratchSlot {
+  void* addr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if unavailable).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
 
 csa_status scratch_for_current_device(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA_ERR_LAUNCH;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_index_scratch) != cudaSuccess || !p) return CSA_ERR_LAUNCH;
-    g_scratch_addr[dev] = p;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    csa::set_last_error(cudaGetErrorString(e));
+    return CSA_ERR_LAUNCH;
   }
-  *out = g_scratch_addr[dev];
+  if (dev < 0 || dev >= kMaxDevices) {
+    csa::set_last_error("csa_index_topk_noalloc: device ordinal beyond the 64 this library tracks");
+    return CSA_ERR_UNSUPPORTED;
+  }
+  // id of the current context (0 before the runtime has made one current:
+  // the lookup below then makes it, and the next call looks up once more)
+  const unsigned long long ctx = current_ctx_id();
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchSlot& slot = g_scratch[dev];
+  if (!slot.addr || slot.ctx_id != ctx) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_index_scratch);
+    if (e != cudaSuccess || !p) {
+      csa::set_last_error(e != cudaSuccess ? cudaGetErrorString(e)
+                                           : "csa_index_topk_noalloc: no device address for the scratch");
+      return CSA_ERR_LAUNCH;
+    }
+    slot.addr = p;
+    slot.ctx_id = ctx;
+  }
+  *out = slot.addr;
   return CSA_OK;
 }
 

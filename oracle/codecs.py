@@ -164,3 +164,39 @@ def mxfp4_decode(packed, scales, n: int) -> np.ndarray:
     sc = ue8m0_decode(scales)
     sc = np.repeat(sc, 32, axis=-1)
     return vals * sc
+
+
+# The 8 non-negative E2M1 values in code order 0..7 (strictly increasing).
+_E2M1_POS = e2m1_decode(np.arange(0, 8))
+E2M1_MAX = 6.0
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """float64 -> E2M1 code (0..15), round to nearest, ties to even,
+    saturating at +-6 (OCP MX v1.0: FP4 has no infinity or NaN, conversions
+    clamp to the largest magnitude).  The sign is kept, so a negative value
+    that rounds to zero becomes -0 (code 8)."""
+    x = np.asarray(x, dtype=np.float64)
+    idx = _nearest_even(_E2M1_POS, np.abs(x))
+    return (idx.astype(np.uint8) | np.where(np.signbit(x), 8, 0).astype(np.uint8)).astype(np.uint8)
+
+
+def mxfp4_encode(x):
+    """float64 [..., n] (n a multiple of 32) -> (packed [..., n/2],
+    scales [..., n/32]) by the OCP MX v1.0 conversion (section 6.3):
+    for each block of 32, the shared exponent is
+        X = floor(log2(max |v|)) - emax_elem,   emax_elem = 2 for E2M1,
+    clamped to the UE8M0 range [-127, 127] (an all-zero block takes
+    X = -127), stored as X + 127; each element becomes the E2M1 code of
+    v / 2^X (nearest even, saturating at +-6: the block's largest magnitude
+    lands in [4, 8) before rounding)."""
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    blk = x.reshape(x.shape[:-1] + (n // 32, 32))
+    amax = np.max(np.abs(blk), axis=-1)
+    with np.errstate(divide="ignore"):
+        X = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2.0, -127.0)
+    X = np.clip(X, -127.0, 127.0)
+    codes = e2m1_encode(blk / np.power(2.0, X)[..., None]).reshape(x.shape)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    return packed, (X + 127).astype(np.uint8)

@@ -191,6 +191,32 @@ def unpack_rows(codes: np.ndarray, scale: np.ndarray, rbits: np.ndarray) -> np.n
 
 
 # ----------------------------------------------------------------------------
+# Index keys and queries in FP4  [kwkr §3.1, §3.4, §4.4; Qiaomu FP4量化感知训练]
+# ----------------------------------------------------------------------------
+
+
+def index_key_compress(a, b, gate, m: int, rope_dims: int, theta: float, eps: float, gamma=None,
+                       e_begin: int = 0, e_end: int | None = None, tok_base: int = 0):
+    """Index keys of entries e in [e_begin, e_end): the same gated
+    compressor as the KV entries (kwkr §3.1: the indexer scores the
+    compressed entries; §3.4: its QK runs in FP4), run over the c_I-dim
+    indexer streams with RoPE on their last ``rope_dims`` dims, then
+    quantised to MXFP4 by the OCP MX conversion.
+
+    Returns (packed [n, c_I/2], scales [n, c_I/32], pos [n])."""
+    keys, pos = compress(a, b, gate, m, rope_dims, theta, eps, gamma, e_begin=e_begin, e_end=e_end,
+                         tok_base=tok_base)
+    packed, scales = codecs.mxfp4_encode(keys)
+    return packed, scales, pos
+
+
+def index_query_quantize(q):
+    """Index queries [..., c_I] -> MXFP4 (packed, scales) by the OCP MX
+    conversion (kwkr §3.4: the indexer QK runs directly in FP4)."""
+    return codecs.mxfp4_encode(q)
+
+
+# ----------------------------------------------------------------------------
 # Lightning Indexer  [Qiaomu 混合注意力机制; kwkr §3.4; WeChat §1.1]
 # ----------------------------------------------------------------------------
 

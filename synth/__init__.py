@@ -346,3 +346,73 @@ def config(name: str, **over):
         kw.update(over)
         return make_workload(kw.pop("seed", 4), p, **kw)
     raise KeyError(name)
+
+
+# ---------------------------------------------------------------------------
+# workload variants (still draws and slices only)
+# ---------------------------------------------------------------------------
+
+
+def with_heads(w, n_h: int):
+    """The workload with only its first ``n_h`` query heads (queries and
+    sinks sliced; nothing else changes)."""
+    p = w["params"]
+    assert n_h <= p.n_h
+    w = dict(w)
+    w["params"] = dataclasses.replace(p, n_h=n_h)
+    w["q"] = np.ascontiguousarray(w["q"][:, :, :n_h])
+    w["sink"] = np.ascontiguousarray(w["sink"][:n_h])
+    return w
+
+
+def _bf16_of(x):
+    return np.asarray(x, np.float32).astype(ml_dtypes.bfloat16).view(np.uint16)
+
+
+def with_wide_rows(w, seed: int, *, scale_log2=(-16.0, 4.0), rope_ratio_log10=(0.0, 4.0),
+                   q_log2=None):
+    """Redraw the FP8 rows' scales and RoPE dims over wide ranges, in storage
+    format: per-row scale 2^u with u ~ U(scale_log2) (codes kept); RoPE dims
+    bf16 of N(0,1) * amax * 10^v, v ~ U(rope_ratio_log10), where amax is the
+    row's decoded non-RoPE amax (so the RoPE/non-RoPE magnitude ratio spans
+    10^v).  With ``q_log2`` the queries are redrawn as
+    bf16 of N(0,1) * 2^u per (query, head), u ~ U(q_log2).  Cache rows and
+    window rows are both redrawn."""
+    p = w["params"]
+    assert p.kv_fmt == FMT_FP8
+    rng = np.random.default_rng(seed)
+    w = dict(w)
+    n_nope = p.d - p.r
+    for key, skey in (("kv", "kv_scale"), ("win", "win_scale")):
+        rows = w[key].copy()
+        shp = rows.shape[:-1]
+        sc = np.exp2(rng.uniform(*scale_log2, size=shp)).astype(np.float32)
+        codes = rows[..., :n_nope].view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+        amax = np.abs(codes).max(axis=-1) * sc
+        ratio = 10.0 ** rng.uniform(*rope_ratio_log10, size=shp)
+        rope = normal_f32(rng, shp + (p.r,)) * (amax * ratio)[..., None].astype(np.float32)
+        rows[..., n_nope:] = _bf16_of(rope).view(np.uint8).reshape(shp + (2 * p.r,))
+        w[key] = rows
+        w[skey] = sc
+    if q_log2 is not None:
+        B, T = w["q"].shape[:2]
+        mag = np.exp2(rng.uniform(*q_log2, size=(B, T, p.n_h, 1))).astype(np.float32)
+        w["q"] = _bf16_of(normal_f32(rng, (B, T, p.n_h, p.d)) * mag)
+    return w
+
+
+_PER_SEQ = ("L", "q_pos0", "a", "b", "gate", "tok_base", "e_begin", "e_end", "kv", "kv_scale", "win",
+            "win_scale", "q_idx", "q_idx_sf", "w_idx", "k_idx", "k_idx_sf", "q")
+
+
+def select_seqs(w, seqs):
+    """The workload restricted to the listed sequences (every per-sequence
+    array sliced along its first axis; capacities unchanged)."""
+    p = w["params"]
+    seqs = list(seqs)
+    out = dict(w)
+    out["params"] = dataclasses.replace(p, B=len(seqs))
+    for k in _PER_SEQ:
+        if k in w and w[k] is not None and not np.isscalar(w[k]):
+            out[k] = np.ascontiguousarray(np.asarray(w[k])[seqs])
+    return out

@@ -10,6 +10,10 @@ Tolerances (stated once, used everywhere):
     RoPE dims within one BF16 ulp of the oracle's value plus 1e-6 absolute
     (the kernel rotates in fp32: a rotated value near zero carries the
     fp32 cancellation error of its unit-size inputs, ~1e-7).
+  * Wide-range attention workloads (row scales, RoPE magnitudes or queries
+    spanning many binades, so outputs are far from unit size): the two
+    BF16/FP8 bounds applied to each head's output divided by the largest
+    magnitude of the oracle's output of that head.
   * Top-k sets: identical (they are unique: ties go to the lower index).
     On fp32 index data (config 0) a mismatch is accepted only where the
     oracle's k-th and (k+1)-th scores are within 1e-5 relative.
@@ -44,6 +48,21 @@ def check_attn(gpu, ref, f32=False, what=""):
     assert mx <= ATTN_MAX_ABS, f"{what}: max abs {mx:.3e} > {ATTN_MAX_ABS}"
     assert mrel <= ATTN_MEAN_REL, f"{what}: mean rel {mrel:.3e} > {ATTN_MEAN_REL}"
     return mx, mrel
+
+
+def check_attn_scaled(gpu, ref, what=""):
+    """check_attn on every (query, head) output normalised by the oracle's
+    largest magnitude of that head (heads with an all-zero oracle output must
+    be all zero)."""
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite GPU output"
+    mag = np.abs(ref).max(axis=-1, keepdims=True)
+    zero = mag[..., 0] == 0
+    assert np.all(gpu[zero] == 0), f"{what}: nonzero output where the oracle's is 0"
+    mag = np.where(mag == 0, 1.0, mag)
+    return check_attn(gpu / mag, ref / mag, what=what)
 
 
 def _mag_index(codes):

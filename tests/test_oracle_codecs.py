@@ -78,3 +78,48 @@ def test_ue8m0_and_mxfp4_layout():
     sc = np.array([127, 128], np.uint8)
     v = codecs.mxfp4_decode(packed, sc, 64)
     assert v[0] == 1.0 and v[1] == 6.0 and v[32] == -3.0 and np.count_nonzero(v) == 3
+
+
+# ---- the OCP MX conversion to MXFP4 (index keys and queries) ---------------
+
+def test_mxfp4_encode_hand_worked_blocks():
+    """Blocks worked by hand from the OCP MX v1.0 conversion rule
+    X = floor(log2 amax) - 2, elements RNE(v / 2^X) on the E2M1 grid
+    {0, .5, 1, 1.5, 2, 3, 4, 6}, saturating."""
+    blk_a = [6.0, 3.0, 1.5, 0.75, -0.25, 5.0, 2.5, -7.0] + [0.0] * 24
+    # amax 7 -> X = floor(2.807) - 2 = 0, scale byte 127
+    # 0.75 ties between .5 and 1 -> 1 (even); -0.25 ties between 0 and .5 ->
+    # -0; 5 ties between 4 and 6 -> 4; 2.5 -> 2; -7 saturates to -6
+    want_a = [0x7, 0x5, 0x3, 0x2, 0x8, 0x6, 0x4, 0xF] + [0x0] * 24
+    blk_b = [0.3, -0.1, 0.05, 0.2] + [0.0] * 28
+    # amax 0.3 -> X = floor(-1.737) - 2 = -4 (byte 123); v * 16 = 4.8 -> 4,
+    # -1.6 -> -1.5, 0.8 -> 1, 3.2 -> 3
+    want_b = [0x6, 0xB, 0x2, 0x5] + [0x0] * 28
+    blk_c = [0.0] * 32  # all zero -> X = -127 (byte 0), codes 0
+    x = np.array([blk_a + blk_b + blk_c + blk_a])
+    packed, scales = codecs.mxfp4_encode(x)
+    assert scales.tolist() == [[127, 123, 0, 127]]
+    nib = np.stack([packed & 0xF, packed >> 4], axis=-1).reshape(1, 128)
+    assert nib[0, :32].tolist() == want_a
+    assert nib[0, 32:64].tolist() == want_b
+    assert nib[0, 64:96].tolist() == [0] * 32
+    # decode: the block's values back on the scaled grid
+    dec = codecs.mxfp4_decode(packed, scales, 128)
+    np.testing.assert_array_equal(dec[0, :8], [6, 3, 1.5, 1, -0.0, 4, 2, -6])
+    np.testing.assert_array_equal(dec[0, 32:36], [0.25, -0.09375, 0.0625, 0.1875])
+
+
+def test_mxfp4_encode_elements_match_library_cast():
+    """Element codes equal ml_dtypes' E2M1 cast (round to nearest even) of
+    v / 2^X, and X is floor(log2 amax) - 2, over values spanning binades."""
+    import ml_dtypes
+    rng = np.random.default_rng(3)
+    y = rng.normal(size=(200, 128)) * np.exp2(rng.uniform(-20, 20, size=(200, 1)))
+    packed, scales = codecs.mxfp4_encode(y)
+    X = scales.astype(np.float64) - 127
+    amax = np.abs(y.reshape(200, 4, 32)).max(axis=-1)
+    np.testing.assert_array_equal(X, np.floor(np.log2(amax)) - 2)
+    ref = (y.reshape(200, 4, 32) / np.exp2(X)[..., None]).astype(np.float32)
+    ref = ref.astype(ml_dtypes.float4_e2m1fn).view(np.uint8).reshape(200, 128) & 0xF
+    nib = np.stack([packed & 0xF, packed >> 4], axis=-1).reshape(200, 128)
+    np.testing.assert_array_equal(nib, ref)

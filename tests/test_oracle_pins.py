@@ -339,3 +339,59 @@ def test_bf16_topk_ranks_collisions_by_index():
 def test_bf16_recall_is_one_when_everything_is_selected():
     w = synth.config("c1", B=1, L=1024)  # n_t = 256 <= k = 512
     assert pipeline.bf16_score_recall(w, [(0, 0)]) == {(0, 0): 1.0}
+
+
+def _f32_index_workload(score_rows, k):
+    """A one-head f32 indexer workload whose scores are given directly:
+    query q = e_0 with weight 1 and key s = (score_s, 0, ...), so that
+    I(t, s) = max(0, score_s).  One query per row of ``score_rows``, each at
+    a position that sees exactly len(row) entries (m = 4)."""
+    n = max(len(r) for r in score_rows)
+    T = len(score_rows)
+    p = synth.Params(B=1, d=128, r=32, m=4, H_I=1, c_I=64, k=k, n_h=1, W=1, tau=1.0,
+                     kv_fmt="f32", idx_fmt="f32", act_fmt="f32")
+    # one key array serves every query: column t of key s holds query t's
+    # score of entry s
+    assert all(len(r) == n for r in score_rows)
+    keys = np.zeros((1, n, 64), np.float32)
+    keys[0, :, :T] = np.asarray(score_rows, np.float32).T   # key s, column t = score of query t
+    q = np.zeros((1, T, 1, 64), np.float32)
+    for t in range(T):
+        q[0, t, 0, t] = 1.0
+    return dict(params=p, T=T, q_pos0=np.array([4 * n - 1], np.int32), Ncap=n, k_idx=keys, q_idx=q,
+                w_idx=np.ones((1, T, 1), np.float32))
+
+
+def test_bf16_recall_hand_worked_half():
+    # FP32 scores 1, 1 + 2^-10, 1 + 2^-9, 0.5: the FP32 top-2 is {1, 2}.  In
+    # BF16 (8 significant bits) the first three all round to 1.0, the tie
+    # goes to the lower indices and the BF16 top-2 is {0, 1}: recall 1/2.
+    w = _f32_index_workload([[1.0, 1.0 + 2.0 ** -10, 1.0 + 2.0 ** -9, 0.5]], k=2)
+    w["q_pos0"] = np.array([15], np.int32)   # n_t = 16 // 4 = 4
+    assert pipeline.index_topk(w)[(0, 0)].tolist() == [1, 2]
+    assert pipeline.index_topk(w, score_fmt="bf16")[(0, 0)].tolist() == [0, 1]
+    assert pipeline.bf16_score_recall(w, [(0, 0)]) == {(0, 0): 0.5}
+
+
+def test_bf16_recall_hand_worked_two_thirds():
+    # scores 3, 2 + 2^-8, 2, 2 + 2^-7, 1 with k = 3: FP32 top-3 = {0, 1, 3};
+    # BF16 keeps 8 significant bits, so near 2 the step is 2^-6: 2 + 2^-8
+    # and 2 + 2^-7 round to 2 and tie with entry 2, which now wins on its
+    # index over entry 3: BF16 top-3 = {0, 1, 2}, recall 2/3.
+    w = _f32_index_workload([[3.0, 2.0 + 2.0 ** -8, 2.0, 2.0 + 2.0 ** -7, 1.0]], k=3)
+    w["q_pos0"] = np.array([19], np.int32)   # n_t = 5
+    assert pipeline.index_topk(w)[(0, 0)].tolist() == [0, 1, 3]
+    assert pipeline.index_topk(w, score_fmt="bf16")[(0, 0)].tolist() == [0, 1, 2]
+    assert pipeline.bf16_score_recall(w, [(0, 0)])[(0, 0)] == pytest.approx(2.0 / 3.0, abs=0)
+
+
+def test_fp8_row_bytes_decode_hand_built():
+    """A stored row built byte by byte from the format definitions: E4M3
+    codes 0x38 (1.0), 0x40 (2.0), 0xB8 (-1.0), 0x01 (2^-9, the smallest
+    subnormal), 0x7E (448, the largest finite), 0x00 (0), times the row
+    scale 0.5; then two BF16 RoPE dims stored little-endian, 0x3F80 (1.0)
+    as bytes 80 3F and 0xC040 (-3.0) as bytes 40 C0."""
+    p = synth.Params(B=1, d=8, r=2, m=4, H_I=1, c_I=64, k=1, n_h=1, W=1, tau=1.0)
+    row = np.array([[0x38, 0x40, 0xB8, 0x01, 0x7E, 0x00, 0x80, 0x3F, 0x40, 0xC0]], np.uint8)
+    got = pipeline.decode_rows(row, np.array([0.5], np.float32), p)
+    np.testing.assert_array_equal(got[0], [0.5, 1.0, -0.5, 2.0 ** -10, 224.0, 0.0, 1.0, -3.0])
