@@ -299,6 +299,79 @@ csa_status csa_index_topk_noalloc(const csa_params* params, const void* q_idx,
                                   int32_t n_max, int32_t* out_idx, int32_t* err,
                                   void* stream);
 
+/* ------------------------------------------------------------------------
+ * Decode-time state  [kwkr 4.4: the KV cache splits into a classical KV
+ *                     cache and a state cache; periodic checkpointing every
+ *                     1024 tokens; kwkr 3.1 / 3.3 for what the state holds]
+ *
+ * A sequence's state beside its compressed entries (the classical cache):
+ *   win     the sliding window's raw tokens, in the cache's row layout,
+ *           token p in ring row p mod win.cap (the `win` of the attention
+ *           calls)
+ *   a, b    the compressor's two stream rings [B][s_cap][d] (act_fmt) and
+ *   gate    its gate logits [B][s_cap][2] fp32, token p in row p mod s_cap;
+ *           s_cap must be a multiple of m and at least T + 2m for every
+ *           append of T tokens (an entry merges its own block of stream a
+ *           with the previous block of stream b).
+ * A checkpoint store keeps the state at multiples P of `every` (a multiple
+ * of m; 1024 on the pages) in n_slots slots per sequence, slot
+ * (P/every - 1) mod n_slots:
+ *   win_rows  [B][n_slots][W][row_bytes], win_scale [B][n_slots][W]
+ *             (CSA_KV_FP8_BF16, else NULL): window rows of positions
+ *             P-W .. P-1 (rows of negative positions stored as zeros)
+ *   a, b      [B][n_slots][m][d] (act_fmt), gate [B][n_slots][m][2]: the
+ *             stream rows of positions P-m .. P-1, all the compressor needs
+ *             to continue at P.
+ * ---------------------------------------------------------------------- */
+typedef struct csa_state {
+  csa_kv win;
+  void* a;
+  void* b;
+  float* gate;
+  int64_t s_cap;
+} csa_state;
+
+typedef struct csa_ckpt {
+  void* win_rows;
+  float* win_scale;
+  void* a;
+  void* b;
+  float* gate;
+  int32_t n_slots;
+  int32_t every;
+} csa_ckpt;
+
+/* csa_state_append: append T tokens of every sequence b at positions
+ * pos0[b] .. pos0[b]+T-1:
+ *   - token tau's KV vector kv_new[b][tau] ([B][T][d], act_fmt, already
+ *     normalised and rotated like the window tokens the attention reads) is
+ *     packed into its window row like a compressed entry (FP8 format:
+ *     scale = amax of the non-RoPE dims / 448, E4M3 codes RNE saturating,
+ *     BF16 RoPE dims);
+ *   - its stream rows a_new[b][tau], b_new[b][tau] ([B][T][d]) and gate
+ *     logits gate_new[b][tau] ([B][T][2]) go into the stream rings;
+ *   - every entry these tokens complete (entries pos0/m .. (pos0+T)/m - 1)
+ *     is compressed from the rings exactly as csa_compress would, into row
+ *     e of `cache` (cache_pos[b][e] = m*e when cache_pos is not NULL);
+ *   - with a checkpoint store (ckpt not NULL), the state at the last
+ *     multiple P of ckpt->every in (pos0, pos0+T] is copied into its slot.
+ * Requirements: win.cap >= window + T - 1 (the attention's own bound),
+ * s_cap a multiple of m with s_cap >= T + 2m.  HCA (m = 128) uses the same
+ * call with its own cache. */
+csa_status csa_state_append(const csa_params* params, const void* kv_new, const void* a_new,
+                            const void* b_new, const float* gate_new, const int32_t* pos0,
+                            int32_t T, csa_state state, csa_kv cache, int32_t* cache_pos,
+                            const csa_ckpt* ckpt, int32_t* err, void* stream);
+
+/* csa_state_restore: put the state checkpointed at pos[b] (a positive
+ * multiple of ckpt->every, still held by its slot) back into the window and
+ * stream rings of sequence b, so that appending can continue at pos[b]
+ * (entries below pos[b]/m must still be in the cache).  A pos[b] that is
+ * not a positive multiple of `every` raises CSA_DEV_ERR_RANGE and leaves
+ * that sequence's rings untouched. */
+csa_status csa_state_restore(const csa_params* params, const int32_t* pos, const csa_ckpt* ckpt,
+                             csa_state state, int32_t* err, void* stream);
+
 /* Human-readable name of a csa_status. */
 const char* csa_status_string(csa_status s);
 

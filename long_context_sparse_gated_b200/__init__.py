@@ -21,7 +21,7 @@ __all__ = [
     "csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn",
     "csa_index_topk_workspace_bytes", "csa_sparse_attn_workspace_bytes",
     "hca_dense_attn_workspace_bytes", "csa_index_topk_noalloc", "csa_index_compress", "csa_index_quantize",
-    "KV_F32", "KV_FP8_BF16", "IDX_F32", "IDX_MXFP4",
+    "CsaState", "CsaCkpt", "csa_state_append", "csa_state_restore", "KV_F32", "KV_FP8_BF16", "IDX_F32", "IDX_MXFP4",
     "ACT_F32", "ACT_BF16", "DEV_ERR_INDEX", "DEV_ERR_RANGE",
 ]
 
@@ -39,7 +39,8 @@ STATUS = {0: "CSA_OK", -1: "CSA_ERR_INVALID", -2: "CSA_ERR_UNSUPPORTED", -3: "CS
 EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_index_topk_workspace_bytes",
            "csa_sparse_attn", "csa_sparse_attn_workspace_bytes", "hca_dense_attn",
            "hca_dense_attn_workspace_bytes", "csa_status_string", "csa_last_error_string",
-           "csa_index_topk_noalloc", "csa_index_compress", "csa_index_quantize"]
+           "csa_index_topk_noalloc", "csa_index_compress", "csa_index_quantize", "csa_state_append",
+           "csa_state_restore"]
 
 
 class CsaError(RuntimeError):
@@ -57,6 +58,17 @@ class CsaParams(ctypes.Structure):
 
 class CsaKv(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("cap", ctypes.c_int64)]
+
+
+class CsaState(ctypes.Structure):
+    _fields_ = [("win", CsaKv), ("a", ctypes.c_void_p), ("b", ctypes.c_void_p), ("gate", ctypes.c_void_p),
+                ("s_cap", ctypes.c_int64)]
+
+
+class CsaCkpt(ctypes.Structure):
+    _fields_ = [("win_rows", ctypes.c_void_p), ("win_scale", ctypes.c_void_p), ("a", ctypes.c_void_p),
+                ("b", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("n_slots", ctypes.c_int32),
+                ("every", ctypes.c_int32)]
 
 
 _lib = None
@@ -95,6 +107,11 @@ def lib(path: str | None = None):
     L.csa_index_compress.restype = _I32
     L.csa_index_quantize.argtypes = [_P, _V, _I64, _V, _V, _V]
     L.csa_index_quantize.restype = _I32
+    L.csa_state_append.argtypes = [_P, _V, _V, _V, _V, _V, _I32, CsaState, CsaKv, _V, ctypes.POINTER(CsaCkpt),
+                                   _V, _V]
+    L.csa_state_append.restype = _I32
+    L.csa_state_restore.argtypes = [_P, _V, ctypes.POINTER(CsaCkpt), CsaState, _V, _V]
+    L.csa_state_restore.restype = _I32
     L.csa_status_string.argtypes = [_I32]
     L.csa_status_string.restype = ctypes.c_char_p
     L.csa_last_error_string.argtypes = []
@@ -180,6 +197,37 @@ def csa_index_quantize(params, x, out, out_sf, stream=None):
     n_rows = x.numel() // params.idx_dim
     st = lib().csa_index_quantize(ctypes.byref(params), _ptr(x), n_rows, _ptr(out), _ptr(out_sf), _stream(stream))
     _check("csa_index_quantize", st)
+
+
+def make_state(win_rows, win_scale, a_ring, b_ring, gate_ring):
+    """csa_state over device tensors: window ring [B, cap, row] (+ scale
+    [B, cap]), stream rings [B, s_cap, d] and gate ring [B, s_cap, 2]."""
+    return CsaState(_kv(win_rows, win_scale), _ptr(a_ring), _ptr(b_ring), _ptr(gate_ring), a_ring.shape[1])
+
+
+def make_ckpt(win_rows, win_scale, a, b, gate, every=1024):
+    """csa_ckpt over device tensors [B, n_slots, W, row], [B, n_slots, W],
+    [B, n_slots, m, d] (x2), [B, n_slots, m, 2]."""
+    return CsaCkpt(_ptr(win_rows), _ptr(win_scale), _ptr(a), _ptr(b), _ptr(gate), win_rows.shape[1], int(every))
+
+
+def csa_state_append(params, kv_new, a_new, b_new, gate_new, pos0, state, cache_rows, cache_scale=None,
+                     cache_pos=None, ckpt=None, err=None, stream=None):
+    """Append T = kv_new.shape[1] tokens per sequence at positions pos0[b]..:
+    window rows, stream rings, the entries they complete, and (with a
+    checkpoint store) the periodic checkpoint."""
+    st = lib().csa_state_append(ctypes.byref(params), _ptr(kv_new), _ptr(a_new), _ptr(b_new), _ptr(gate_new),
+                                _ptr(pos0), int(kv_new.shape[1]), state, _kv(cache_rows, cache_scale),
+                                _ptr(cache_pos), None if ckpt is None else ctypes.byref(ckpt), _ptr(err),
+                                _stream(stream))
+    _check("csa_state_append", st)
+
+
+def csa_state_restore(params, pos, ckpt, state, err=None, stream=None):
+    """Put the state checkpointed at pos[b] back into the rings."""
+    st = lib().csa_state_restore(ctypes.byref(params), _ptr(pos), ctypes.byref(ckpt), state, _ptr(err),
+                                 _stream(stream))
+    _check("csa_state_restore", st)
 
 
 def csa_index_topk_workspace_bytes(params, T, n_max):

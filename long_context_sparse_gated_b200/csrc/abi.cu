@@ -242,6 +242,56 @@ csa_status hca_dense_attn(const csa_params* p, const void* q, csa_kv cache, csa_
                    stream);
 }
 
+static csa_status check_state(const csa_params* p, const csa_state& s, int32_t T) {
+  csa_status st = check_kv(p, s.win);
+  if (st != CSA_OK) return st;
+  if (!s.a || !s.b || !s.gate) return CSA_ERR_INVALID;
+  for (const void* ptr : {(const void*)s.a, (const void*)s.b, (const void*)s.gate})
+    if (!aligned16(ptr)) return CSA_ERR_ALIGN;
+  if (s.s_cap < (int64_t)T + 2 * p->m || s.s_cap % p->m) return CSA_ERR_INVALID;
+  if (s.win.cap < (int64_t)p->window + T - 1) return CSA_ERR_INVALID;
+  return CSA_OK;
+}
+
+static csa_status check_ckpt(const csa_params* p, const csa_ckpt& c) {
+  if (c.n_slots < 1 || c.every < p->m || c.every % p->m) return CSA_ERR_INVALID;
+  if (!c.win_rows || !c.a || !c.b || !c.gate) return CSA_ERR_INVALID;
+  if (p->kv_fmt == CSA_KV_FP8_BF16 && !c.win_scale) return CSA_ERR_INVALID;
+  for (const void* ptr : {(const void*)c.win_rows, (const void*)c.a, (const void*)c.b, (const void*)c.gate})
+    if (!aligned16(ptr)) return CSA_ERR_ALIGN;
+  if (c.win_scale && !aligned16(c.win_scale)) return CSA_ERR_ALIGN;
+  return CSA_OK;
+}
+
+csa_status csa_state_append(const csa_params* p, const void* kv_new, const void* a_new, const void* b_new,
+                            const float* gate_new, const int32_t* pos0, int32_t T, csa_state state, csa_kv cache,
+                            int32_t* cache_pos, const csa_ckpt* ckpt, int32_t* err, void* stream) {
+  csa_status s = check_params(p);
+  if (s != CSA_OK) return s;
+  if (p->window < 1 || p->window > 1024) return CSA_ERR_UNSUPPORTED;
+  if (T < 1 || T > 65535 || !kv_new || !a_new || !b_new || !gate_new || !pos0) return CSA_ERR_INVALID;
+  for (const void* ptr : {kv_new, a_new, b_new, (const void*)gate_new, (const void*)pos0})
+    if (!aligned16(ptr)) return CSA_ERR_ALIGN;
+  if (cache_pos && !aligned16(cache_pos)) return CSA_ERR_ALIGN;
+  if ((s = check_state(p, state, T)) != CSA_OK) return s;
+  if ((s = check_kv(p, cache)) != CSA_OK) return s;
+  if (ckpt && (s = check_ckpt(p, *ckpt)) != CSA_OK) return s;
+  return launched(csa::launch_state_append(*p, kv_new, a_new, b_new, gate_new, pos0, T, state, cache, cache_pos, ckpt,
+                                           err, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+csa_status csa_state_restore(const csa_params* p, const int32_t* pos, const csa_ckpt* ckpt, csa_state state,
+                             int32_t* err, void* stream) {
+  csa_status s = check_params(p);
+  if (s != CSA_OK) return s;
+  if (p->window < 1 || p->window > 1024) return CSA_ERR_UNSUPPORTED;
+  if (!pos || !ckpt) return CSA_ERR_INVALID;
+  if (!aligned16(pos)) return CSA_ERR_ALIGN;
+  if ((s = check_state(p, state, 1)) != CSA_OK) return s;
+  if ((s = check_ckpt(p, *ckpt)) != CSA_OK) return s;
+  return launched(csa::launch_state_restore(*p, pos, *ckpt, state, err, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char* csa_last_error_string(void) { return g_last_error; }
 
 const char* csa_status_string(csa_status s) {

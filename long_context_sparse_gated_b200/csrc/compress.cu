@@ -25,7 +25,7 @@ __global__ void __launch_bounds__(1024) compress_kernel(
     const float* __restrict__ gate, int64_t S, const int32_t* __restrict__ tok_base,
     const int32_t* __restrict__ e_begin, const int32_t* __restrict__ e_end,
     const float* __restrict__ norm_w, uint8_t* __restrict__ rows, float* __restrict__ scale,
-    int64_t cap, int32_t* __restrict__ out_pos, int32_t* __restrict__ err) {
+    int64_t cap, int32_t* __restrict__ out_pos, int32_t* __restrict__ err, int64_t ring, int T_new) {
   extern __shared__ float smem[];
   const int m = p.m, d = p.d, r = p.r;
   const int quads = d >> 2;
@@ -37,13 +37,19 @@ __global__ void __launch_bounds__(1024) compress_kernel(
   pdl_wait();
   pdl_trigger();
   const int bs = blockIdx.y;
-  const int64_t e = (int64_t)e_begin[bs] + blockIdx.x;
-  if (e >= e_end[bs]) return;
-  const int64_t base = tok_base[bs];
-  const int64_t ia0 = (int64_t)m * e - base;
+  // Linear buffers: entries [e_begin, e_end), token p at row p - tok_base.
+  // Ring buffers (ring > 0, the decode state): e_begin holds the position
+  // of the first of T_new appended tokens; the entries they complete are
+  // [pos0/m, (pos0+T_new)/m), and token p sits at row p mod ring.
+  const int64_t eb = ring ? (int64_t)e_begin[bs] / m : (int64_t)e_begin[bs];
+  const int64_t ee = ring ? ((int64_t)e_begin[bs] + T_new) / m : (int64_t)e_end[bs];
+  const int64_t e = eb + blockIdx.x;
+  if (e >= ee) return;
+  const int64_t base = ring ? 0 : tok_base[bs];
   const int nb = e > 0 ? m : 0;
-  const int64_t ib0 = (int64_t)m * (e - 1) - base;
-  if (ia0 < 0 || ia0 + m > S || (nb && ib0 < 0) || e >= cap) {
+  const int64_t ia0 = ring ? ((int64_t)m * e) % ring : (int64_t)m * e - base;
+  const int64_t ib0 = ring ? (e > 0 ? ((int64_t)m * (e - 1)) % ring : 0) : (int64_t)m * (e - 1) - base;
+  if (e >= cap || (!ring && (ia0 < 0 || ia0 + m > S || (nb && ib0 < 0)))) {
     if (threadIdx.x == 0) raise_err(err, CSA_DEV_ERR_RANGE);
     return;
   }
@@ -202,7 +208,29 @@ cudaError_t launch_compress(const csa_params& p, const void* a, const void* b, c
   auto kfn = f32 ? (kv32 ? compress_kernel<true, kOutF32> : compress_kernel<true, kOutFp8>)
                  : (kv32 ? compress_kernel<false, kOutF32> : compress_kernel<false, kOutFp8>);
   cudaError_t e = launch_pdl(kfn, grid, dim3(threads), smem, st, p, a, b, gate, S, tok_base, e_begin, e_end, norm_w,
-                             rows, out.scale, out.cap, out_pos, err);
+                             rows, out.scale, out.cap, out_pos, err, (int64_t)0, 0);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// The entries completed by T_new tokens appended at pos0[b], read from the
+// stream rings (token p at row p mod ring).
+cudaError_t launch_compress_ring(const csa_params& p, const void* a, const void* b, const float* gate, int64_t ring,
+                                 const int32_t* pos0, int T_new, const csa_kv& out, int32_t* out_pos, int32_t* err,
+                                 cudaStream_t st) {
+  const int quads = p.d / 4;
+  int threads = p.m >= 64 ? 1024 : 256;
+  if (threads < quads) threads = quads;
+  const int G = threads / quads;
+  const size_t smem = (size_t)(2 * p.m + G * p.d) * sizeof(float);
+  const int max_entries = (T_new + p.m - 1) / p.m;  // block ends among T_new consecutive tokens
+  dim3 grid(max_entries, p.B);
+  const bool f32 = p.act_fmt == CSA_ACT_F32, kv32 = p.kv_fmt == CSA_KV_F32;
+  auto kfn = f32 ? (kv32 ? compress_kernel<true, kOutF32> : compress_kernel<true, kOutFp8>)
+                 : (kv32 ? compress_kernel<false, kOutF32> : compress_kernel<false, kOutFp8>);
+  cudaError_t e = launch_pdl(kfn, grid, dim3(threads), smem, st, p, a, b, gate, ring, (const int32_t*)nullptr, pos0,
+                             (const int32_t*)nullptr, (const float*)nullptr, reinterpret_cast<uint8_t*>(out.rows),
+                             out.scale, out.cap, out_pos, err, ring, T_new);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -225,7 +253,7 @@ cudaError_t launch_index_compress(const csa_params& p, int rope_dims, const void
   auto kfn = p.act_fmt == CSA_ACT_F32 ? compress_kernel<true, kOutMxfp4> : compress_kernel<false, kOutMxfp4>;
   cudaError_t e = launch_pdl(kfn, grid, dim3(threads), smem, st, q, a, b, gate, S, tok_base, e_begin, e_end, norm_w,
                              reinterpret_cast<uint8_t*>(k_idx), reinterpret_cast<float*>(k_idx_sf), k_cap,
-                             (int32_t*)nullptr, err);
+                             (int32_t*)nullptr, err, (int64_t)0, 0);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

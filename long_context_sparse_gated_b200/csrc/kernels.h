@@ -45,6 +45,18 @@ cudaError_t launch_index_compress(const csa_params& p, int rope_dims, const void
 cudaError_t launch_index_quantize(const csa_params& p, const void* x, int64_t n_rows, void* out, uint8_t* out_sf,
                                   cudaStream_t st);
 
+cudaError_t launch_compress_ring(const csa_params& p, const void* a, const void* b, const float* gate, int64_t ring,
+                                 const int32_t* pos0, int T_new, const csa_kv& out, int32_t* out_pos, int32_t* err,
+                                 cudaStream_t st);
+
+cudaError_t launch_state_append(const csa_params& p, const void* kv_new, const void* a_new, const void* b_new,
+                                const float* gate_new, const int32_t* pos0, int T, const csa_state& s,
+                                const csa_kv& cache, int32_t* cache_pos, const csa_ckpt* ck, int32_t* err,
+                                cudaStream_t st);
+
+cudaError_t launch_state_restore(const csa_params& p, const int32_t* pos, const csa_ckpt& ck, const csa_state& s,
+                                 int32_t* err, cudaStream_t st);
+
 cudaError_t launch_index_scores(const csa_params& p, const void* q_idx, const uint8_t* q_sf,
                                 const float* w, const void* k_idx, const uint8_t* k_sf,
                                 int64_t k_cap, const int32_t* q_pos0, int T, float* scores,

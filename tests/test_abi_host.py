@@ -55,6 +55,14 @@ r['k_too_big'] = st('csa_index_topk', ctypes.byref(m.make_params(B=2, d=512, r=6
 r['n_max_gt_cap'] = st('csa_index_topk', ctypes.byref(P), A, A, A, A, A, 100, A, 1, 101, A, A, 1 << 30, None, None)
 r['null_sink'] = st('csa_sparse_attn', ctypes.byref(P), A, kv, A, m.CsaKv(A, A, 128), None, A, 1, A, A, 1 << 30, None, None)
 r['small_window'] = st('csa_sparse_attn', ctypes.byref(P), A, kv, A, m.CsaKv(A, A, 64), A, A, 1, A, A, 1 << 30, None, None)
+state_small = m.CsaState(m.CsaKv(A, A, 256), A, A, A, 8)      # s_cap 8 < T + 2m
+r['state_small_ring'] = st('csa_state_append', ctypes.byref(P), A, A, A, A, A, 1, state_small, kv, None, None, None, None)
+state_ok = m.CsaState(m.CsaKv(A, A, 256), A, A, A, 64)
+ck_bad = m.CsaCkpt(A, A, A, A, A, 2, 1022)                       # period not a multiple of m
+r['ckpt_period'] = st('csa_state_append', ctypes.byref(P), A, A, A, A, A, 1, state_ok, kv, None, ctypes.byref(ck_bad), None, None)
+r['restore_null'] = st('csa_state_restore', ctypes.byref(P), A, None, state_ok, None, None)
+r['quant_dim'] = st('csa_index_quantize', ctypes.byref(m.make_params(B=1, d=512, r=64, m=4, idx_dim=96)), A, 8, A, A, None)
+r['ikc_rope'] = st('csa_index_compress', ctypes.byref(P), A, A, A, 8, A, A, A, 1, 6, None, A, A, 10, None, None)
 r['ws_bytes'] = L.csa_index_topk_workspace_bytes(ctypes.byref(P), 1, 32768)
 r['attn_ws'] = L.csa_sparse_attn_workspace_bytes(ctypes.byref(P), 1)
 r['name'] = L.csa_status_string(-4).decode()
@@ -76,6 +84,11 @@ def test_host_validation_codes():
     assert r["n_max_gt_cap"] == -1
     assert r["null_sink"] == -1
     assert r["small_window"] == -1
+    assert r["state_small_ring"] == -1
+    assert r["ckpt_period"] == -1
+    assert r["restore_null"] == -1
+    assert r["quant_dim"] == -2
+    assert r["ikc_rope"] == -2
     assert r["ws_bytes"] == 2 * 32768 * 4 + 2 * 4096 * 4  # scores + per-query histograms
     assert r["attn_ws"] > 0
     assert r["name"] == "CSA_ERR_WORKSPACE"

@@ -28,9 +28,9 @@ def _lib():
     build.build()
 
 
-def _params(idx_dim, act, m=4):
+def _params(idx_dim, act, m=4, B=1):
     from long_context_sparse_gated_b200 import ACT_BF16, ACT_F32, make_params
-    return make_params(B=1, d=512, r=64, m=m, n_idx_heads=64, idx_dim=idx_dim,
+    return make_params(B=B, d=512, r=64, m=m, n_idx_heads=64, idx_dim=idx_dim,
                        act_fmt=ACT_BF16 if act == "bf16" else ACT_F32)
 
 
@@ -97,7 +97,7 @@ def test_index_compress_matches_oracle(act, c, m, rope):
     k = torch.zeros((B, k_cap, c // 2), dtype=torch.uint8, device="cuda")
     ksf = torch.zeros((B, k_cap, c // 32), dtype=torch.uint8, device="cuda")
     err = torch.zeros(4, dtype=torch.int32, device="cuda")
-    p = _params(c, act, m)
+    p = _params(c, act, m, B=B)
     csa_index_compress(p, ta, tb, torch.from_numpy(gate).cuda(), zeros, zeros, e_end, n_ent, rope, k, ksf, err=err)
     torch.cuda.synchronize()
     assert int(err[0]) == 0

@@ -395,3 +395,37 @@ def test_fp8_row_bytes_decode_hand_built():
     row = np.array([[0x38, 0x40, 0xB8, 0x01, 0x7E, 0x00, 0x80, 0x3F, 0x40, 0xC0]], np.uint8)
     got = pipeline.decode_rows(row, np.array([0.5], np.float32), p)
     np.testing.assert_array_equal(got[0], [0.5, 1.0, -0.5, 2.0 ** -10, 224.0, 0.0, 1.0, -3.0])
+
+
+# ---- decode-time state (oracle.state) --------------------------------------
+
+def test_state_checkpoint_positions_brute_force():
+    from oracle import state
+    for a0 in range(0, 3000, 37):
+        for T in (1, 5, 1024, 1500):
+            ref = [P for P in range(a0 + 1, a0 + T + 1) if P % 1024 == 0]
+            assert state.checkpoints(a0, a0 + T, 1024) == ref
+
+
+def test_state_window_and_stream_extent():
+    from oracle import state
+    rng = np.random.default_rng(5)
+    kv = rng.normal(size=(300, 8))
+    ws = state.window_state(kv, 200, 128, 2, "fp8")
+    assert sorted(ws) == list(range(72, 200))
+    c, s, rb = ws[100]
+    # a window row is the token's own vector in the entry layout
+    np.testing.assert_allclose(csa.unpack_rows(c[None], np.array([s]), rb[None])[0], kv[100], rtol=0.07, atol=1e-2)
+    assert sorted(state.window_state(kv, 50, 128, 2, "fp8")) == list(range(50))
+    ss = state.stream_state(kv, kv, kv[:, :2], 256, 4)
+    assert sorted(ss) == [252, 253, 254, 255]
+
+
+def test_state_entries_after_are_the_complete_blocks():
+    from oracle import state
+    rng = np.random.default_rng(6)
+    a, b, g = rng.normal(size=(23, 8)), rng.normal(size=(23, 8)), rng.normal(size=(23, 2))
+    ent, pos = state.entries_after(a, b, g, 23, 4, 2, 1e4, 1e-6)
+    assert pos.tolist() == [0, 4, 8, 12, 16]          # entry 5 would need token 23
+    ref, _ = csa.compress(a[:20], b[:20], g[:20], 4, 2, 1e4, 1e-6)
+    np.testing.assert_array_equal(ent, ref)
