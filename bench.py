@@ -118,6 +118,39 @@ def index_flops(w):
 
 FP4_OVER_BF16 = 4.0  # nominal dense ratio of B200's FP4 and BF16 tensor rates (9 / 2.25 PFLOP/s)
 
+_PEAK_CACHE = {}
+
+
+def probe_tensor_peak(kind):
+    """Dense tcgen05.mma throughput measured live on this GPU by the probe
+    library (every SM issuing back-to-back M=128, N=256 MMAs; best of 5
+    launches): kind "mxf4" (E2M1, block-scaled) or "bf16".  TFLOP/s, or None
+    if the probe fails."""
+    if kind in _PEAK_CACHE:
+        return _PEAK_CACHE[kind]
+    val = None
+    try:
+        import ctypes
+        from long_context_sparse_gated_b200 import build
+        L = ctypes.CDLL(build.build_peak())
+        L.csa_peak_mma_tflops.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.csa_peak_mma_tflops.restype = ctypes.c_double
+        v = L.csa_peak_mma_tflops(0 if kind == "mxf4" else 1, 20000, 5)
+        val = v if v > 0 else None
+    except Exception:
+        val = None
+    _PEAK_CACHE[kind] = val
+    return val
+
+
+def fp4_peak(bf16_peak, bf16_src):
+    """The MXFP4 dense peak: measured by the probe, else the BF16 peak times
+    the nominal ratio (said so in the source string)."""
+    v = probe_tensor_peak("mxf4")
+    if v is not None:
+        return v, "measured live: tcgen05.mma kind::mxf4 M=128 N=256 K=64, all SMs, best of 5 (bench.py probe)"
+    return bf16_peak * FP4_OVER_BF16, f"{bf16_src} bf16 x {FP4_OVER_BF16:g} (nominal fp4:bf16)"
+
 
 def dominant_roofline(w, kmean_ms, idx_bytes, step_bytes, hbm, bf16, traffic):
     """Roofline entry of the step's dominant call.  hbm = (GB/s, source) and
@@ -136,17 +169,18 @@ def dominant_roofline(w, kmean_ms, idx_bytes, step_bytes, hbm, bf16, traffic):
     hbm_ach = dom_bytes / sec / 1e9
     if p.k > 0:
         fl = index_flops(w)
-        fp4_peak = bf16_peak * FP4_OVER_BF16
+        fp4_pk, fp4_src = fp4_peak(bf16_peak, bf16_src)
         fp4_ach = fl / sec / 1e12
         if w["T"] <= 4:
             return {"bound": "hbm", "kernel": "csa_index_topk", "achieved": hbm_ach, "peak": hbm_peak,
                     "unit": "GB/s", "frac": hbm_ach / hbm_peak, "peak_source": hbm_src, "traffic": traffic,
                     "frac_vs_8tbs_datasheet": hbm_ach / 8000.0,
                     "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean_ms,
-                    "fp4_tflops": fp4_ach, "fp4_frac": fp4_ach / fp4_peak}
-        return {"bound": "tensor", "kernel": "csa_index_topk", "achieved": fp4_ach, "peak": fp4_peak,
-                "unit": "TFLOP/s", "frac": fp4_ach / fp4_peak,
-                "peak_source": f"{bf16_src} bf16 x {FP4_OVER_BF16:g} (nominal fp4:bf16)", "traffic": traffic,
+                    "fp4_tflops": fp4_ach, "fp4_peak": fp4_pk, "fp4_frac": fp4_ach / fp4_pk,
+                    "fp4_peak_source": fp4_src}
+        return {"bound": "tensor", "kernel": "csa_index_topk", "achieved": fp4_ach, "peak": fp4_pk,
+                "unit": "TFLOP/s", "frac": fp4_ach / fp4_pk,
+                "peak_source": fp4_src, "traffic": traffic,
                 "algorithmic_flops_per_launch": fl, "launch_ms": kmean_ms,
                 "hbm_achieved_gbs": hbm_ach, "hbm_frac": hbm_ach / hbm_peak}
     fl = algorithmic_flops(w)
@@ -165,8 +199,9 @@ def step_roofline_entry(w, ms_per_step, step_bytes, hbm_peak, bf16_peak):
     sec = ms_per_step * 1e-3
     gbs = step_bytes / sec / 1e9
     fl_i, fl_a = index_flops(w), algorithmic_flops(w)
+    fp4_pk = fp4_peak(bf16_peak, "")[0]
     return {"algorithmic_bytes": step_bytes, "achieved_gbs": gbs, "frac": gbs / hbm_peak,
-            "index_fp4_tflops": fl_i / sec / 1e12, "index_fp4_frac": fl_i / sec / 1e12 / (bf16_peak * FP4_OVER_BF16),
+            "index_fp4_tflops": fl_i / sec / 1e12, "index_fp4_frac": fl_i / sec / 1e12 / fp4_pk,
             "attn_tflops": fl_a / sec / 1e12, "attn_bf16_frac": fl_a / sec / 1e12 / bf16_peak}
 
 
@@ -431,6 +466,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch every call from the host (no CUDA graphs)")
     ap.add_argument("--copies", type=int, default=0,
                     help="device copies rotated in the timed loop (0: enough to exceed 3x L2)")
+    ap.add_argument("--extra-configs", default="c2,c3,c4",
+                    help="with --config c1 on one GPU: the other workloads measured into the same line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -449,17 +486,44 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     from long_context_sparse_gated_b200 import build, lib
-    from long_context_sparse_gated_b200.runner import STEP_INPUTS, DeviceWorkload
     if rank == 0 or world == 1:
         build.build()
     if world > 1:
         dist.barrier()
     lib()
 
-    w = synth.config(args.config, seed=rank_seed(args.config, rank))
+    names = [args.config]
+    if world == 1 and args.config == "c1":
+        names += [c for c in args.extra_configs.split(",") if c and c != args.config]
+    lines = {}
+    for name in names:
+        lines[name] = run_config(name, args, world, rank, local)
+        torch.cuda.empty_cache()
+    if rank == 0:
+        line = lines[names[0]]
+        if len(names) > 1:
+            # the other workloads of the same metric, each measured the same
+            # way (its own roofline, clocks, end-to-end and CPU baseline)
+            line["configs"] = {n: lines[n] for n in names[1:]}
+        line["tensor_peaks_measured"] = {"mxf4_tflops": probe_tensor_peak("mxf4"),
+                                         "bf16_tflops": probe_tensor_peak("bf16"),
+                                         "how": "tcgen05.mma M=128 N=256 back to back from one thread per SM, all SMs, "
+                                                "best of 5 launches of 20000 MMAs (burst)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_config(config, args, world, rank, local):
+    """Measure one workload; rank 0 returns its JSON entry, others None."""
+    import torch
+    import torch.distributed as dist
+    from long_context_sparse_gated_b200.runner import STEP_INPUTS, DeviceWorkload
+
+    w = synth.config(config, seed=rank_seed(config, rank))
     step_bytes, idx_bytes = algorithmic_bytes(w)
     n_copies = max(1, int(np.ceil(3 * L2_BYTES / step_bytes)))
-    if args.config == "c4":
+    if config == "c4":
         n_copies = 1  # prefill touches far more than L2 per step
     if args.copies > 0:
         n_copies = args.copies
@@ -649,20 +713,19 @@ def main():
     err = int(sum(d.err_bits() for d in dws))
 
     if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
-        return
+        del dws
+        return None
     ms_per_step = ms / args.steps
     value = job_value(world, queries, ms_per_step)
     peak, peak_kind = measured_peaks()
     roofline = dominant_roofline(w, kmean, idx_bytes, step_bytes, (peak, peak_kind), measured_tensor_peak(),
-                                 recorded_traffic(f"csa_index_topk@{args.config}") if p.k > 0 else None)
+                                 recorded_traffic(f"csa_index_topk@{config}") if p.k > 0 else None)
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8/bf16 storage, mxfp4 indexer, fp32 accumulate" if p.kv_fmt == "fp8" else "f32",
         "data": "synthetic",
-        "config": {"workload": CONFIG_NAMES[args.config], "name": args.config, "batch": p.B,
+        "config": {"workload": CONFIG_NAMES[config], "name": config, "batch": p.B,
                    "context": int(w["L"].max()), "queries_per_step": queries,
                    "l2": f"inputs larger than L2: {n_copies} device copies rotated, {n_copies * step_bytes / 2**20:.0f} MiB per cycle"},
         "gpu_launches": args.steps * (kernels_per_step if kernels_per_step is not None else launches_per_step(w)),
@@ -676,10 +739,9 @@ def main():
         "device_err_bits": err,
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline_entry(w, args.config)
-    print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+        line["cpu_baseline"] = cpu_baseline_entry(w, config)
+    del dws
+    return line
 
 
 if __name__ == "__main__":

@@ -83,6 +83,8 @@ typedef int32_t csa_status;
 #define CSA_IDX_MXFP4 1
 #define CSA_ACT_F32 0
 #define CSA_ACT_BF16 1
+#define CSA_SCORE_F32 0  /* index scores kept in fp32 before selection      */
+#define CSA_SCORE_BF16 1 /* index scores rounded to BF16 (RNE) before it   */
 
 /* Layer configuration (host struct, plain old data).
  *   B            sequences in the batch
@@ -98,6 +100,10 @@ typedef int32_t csa_status;
  *   rope_theta     RoPE base (pair j of the last r dims turns by
  *                  pos * theta^(-2j/r))
  *   eps            RMSNorm epsilon
+ *   score_fmt      CSA_SCORE_F32 or CSA_SCORE_BF16: the precision of the
+ *                  index scores the top-k selector ranks ([kwkr 4.4]: the
+ *                  scores are quantised from FP32 to BF16 before the
+ *                  selector; ties after rounding go to the lower index)
  */
 typedef struct csa_params {
   int32_t B, d, r, m;
@@ -105,6 +111,7 @@ typedef struct csa_params {
   int32_t topk, n_heads, window;
   int32_t kv_fmt, idx_fmt, act_fmt;
   float softmax_scale, rope_theta, eps;
+  int32_t score_fmt;
 } csa_params;
 
 /* A KV-row buffer: the compressed-entry cache, or the raw-token window ring.

@@ -22,13 +22,14 @@ __all__ = [
     "csa_index_topk_workspace_bytes", "csa_sparse_attn_workspace_bytes",
     "hca_dense_attn_workspace_bytes", "csa_index_topk_noalloc", "csa_index_compress", "csa_index_quantize",
     "CsaState", "CsaCkpt", "csa_state_append", "csa_state_restore", "KV_F32", "KV_FP8_BF16", "IDX_F32", "IDX_MXFP4",
-    "ACT_F32", "ACT_BF16", "DEV_ERR_INDEX", "DEV_ERR_RANGE",
+    "ACT_F32", "ACT_BF16", "SCORE_F32", "SCORE_BF16", "DEV_ERR_INDEX", "DEV_ERR_RANGE",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcsa.so")
 
 KV_F32, KV_FP8_BF16 = 0, 1
+SCORE_F32, SCORE_BF16 = 0, 1
 IDX_F32, IDX_MXFP4 = 0, 1
 ACT_F32, ACT_BF16 = 0, 1
 DEV_ERR_INDEX, DEV_ERR_RANGE = 1, 2
@@ -53,7 +54,8 @@ class CsaParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "d", "r", "m", "n_idx_heads", "idx_dim", "topk", "n_heads", "window",
                  "kv_fmt", "idx_fmt", "act_fmt")] + \
-               [(n, ctypes.c_float) for n in ("softmax_scale", "rope_theta", "eps")]
+               [(n, ctypes.c_float) for n in ("softmax_scale", "rope_theta", "eps")] + \
+               [("score_fmt", ctypes.c_int32)]
 
 
 class CsaKv(ctypes.Structure):
@@ -125,9 +127,9 @@ def lib(path: str | None = None):
 
 def make_params(*, B, d, r, m, n_idx_heads=1, idx_dim=64, topk=1, n_heads=1, window=1,
                 kv_fmt=KV_FP8_BF16, idx_fmt=IDX_MXFP4, act_fmt=ACT_BF16, softmax_scale=1.0,
-                rope_theta=1e4, eps=1e-6) -> CsaParams:
+                rope_theta=1e4, eps=1e-6, score_fmt=SCORE_F32) -> CsaParams:
     return CsaParams(B, d, r, m, n_idx_heads, idx_dim, topk, n_heads, window, kv_fmt, idx_fmt,
-                     act_fmt, softmax_scale, rope_theta, eps)
+                     act_fmt, softmax_scale, rope_theta, eps, score_fmt)
 
 
 def _ptr(t):

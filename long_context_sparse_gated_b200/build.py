@@ -40,6 +40,7 @@ def up_to_date() -> bool:
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
+        build_peak()
         return LIB
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
@@ -67,7 +68,26 @@ def build(force: bool = False, verbose: bool = False) -> str:
         f.write("\n".join(log))
     if verbose:
         print("\n".join(log))
+    build_peak(force=force)
     return LIB
+
+
+PEAK_LIB = os.path.join(PKG, "peak", "libcsa_peak.so")
+
+
+def build_peak(force: bool = False) -> str:
+    """The benchmark's tensor-throughput probe (not part of libcsa)."""
+    src = os.path.join(PKG, "peak", "mma_peak.cu")
+    deps = [src, os.path.join(PKG, "csrc", "sm100.cuh"), __file__]
+    if not force and os.path.exists(PEAK_LIB) and all(os.path.getmtime(f) <= os.path.getmtime(PEAK_LIB) for f in deps):
+        return PEAK_LIB
+    tmp = PEAK_LIB + ".tmp"
+    cmd = [NVCC, *ARCH, "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", src, "-o", tmp, "-lcudart"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
+    os.replace(tmp, PEAK_LIB)
+    return PEAK_LIB
 
 
 if __name__ == "__main__":

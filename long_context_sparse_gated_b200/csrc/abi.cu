@@ -77,16 +77,22 @@ csa_status compress_impl(const csa_params* p, const void* a, const void* b, cons
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
-// Index workspace: fp32 scores [B*T][ld] (ld = n_max rounded up to 32),
-// then, for decode-sized batches, a 4096-bin histogram per query.
+// Index workspace: scores [B*T][ld] (ld = n_max rounded up to 32; fp32, or
+// BF16 with CSA_SCORE_BF16), then, for decode-sized batches, the region the
+// call clears (4096-bin histogram, tie count and 256-bin second-level
+// histogram per query) and, for rows over 32768 entries, selection bitmaps
+// and tie lists.
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
 size_t scores_bytes(const csa_params* p, int32_t T, int32_t n_max) {
-  size_t b = (size_t)p->B * (size_t)T * (size_t)csa::topk_scores_ld(n_max) * sizeof(float);
-  return (b + 255) & ~(size_t)255;
+  const size_t el = p->score_fmt == CSA_SCORE_BF16 ? 2 : 4;
+  return round256((size_t)p->B * (size_t)T * (size_t)csa::topk_scores_ld(n_max) * el);
 }
 
 size_t index_ws_bytes(const csa_params* p, int32_t T, int32_t n_max) {
   size_t b = scores_bytes(p, T, n_max);
-  if (csa::topk_use_hist(p->B * T)) b += csa::topk_hist_bytes(p->B * T) + csa::topk_cand_bytes(p->B * T, n_max);
+  const int nq = p->B * T;
+  if (csa::topk_use_hist(nq)) b += round256(csa::topk_zero_bytes(nq)) + csa::topk_extra_bytes(nq, n_max);
   return b;
 }
 
@@ -159,6 +165,7 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
   if (p->n_idx_heads < 1 || p->n_idx_heads > 64) return CSA_ERR_UNSUPPORTED;
   if (p->idx_dim != 64 && p->idx_dim != 128) return CSA_ERR_UNSUPPORTED;
   if (p->topk < 1 || p->topk > 2048) return CSA_ERR_UNSUPPORTED;
+  if (p->score_fmt != CSA_SCORE_F32 && p->score_fmt != CSA_SCORE_BF16) return CSA_ERR_UNSUPPORTED;
   if (!q_idx || !w || !k_idx || !q_pos0 || !out_idx || T < 1 || n_max < 0 || k_cap < 1 ||
       n_max > k_cap)
     return CSA_ERR_INVALID;
@@ -171,13 +178,16 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
   if (ws_bytes < need || (need && !ws)) return CSA_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return CSA_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float* scores = reinterpret_cast<float*>(ws);
+  void* scores = ws;
   const int ld = csa::topk_scores_ld(n_max);
+  const int nq = p->B * T;
   const bool tc = csa::index_scores_tc_supported(*p, k_cap, q_idx, q_idx_sf, k_idx, k_idx_sf);
   uint32_t* hist = nullptr;
-  if (tc && csa::topk_use_hist(p->B * T) && n_max > p->topk) {
+  void* extra = nullptr;
+  if (tc && csa::topk_use_hist(nq) && n_max > p->topk) {
     hist = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + scores_bytes(p, T, n_max));
-    cudaError_t e = cudaMemsetAsync(hist, 0, csa::topk_hist_bytes(p->B * T), st);
+    extra = reinterpret_cast<char*>(hist) + round256(csa::topk_zero_bytes(nq));
+    cudaError_t e = cudaMemsetAsync(hist, 0, csa::topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return launched(e);
   }
   if (n_max > 0) {
@@ -190,8 +200,8 @@ csa_status csa_index_topk(const csa_params* p, const void* q_idx, const uint8_t*
                                    n_max, err, st);
     if (e != cudaSuccess) return launched(e);
   }
-  void* cand = hist ? reinterpret_cast<char*>(hist) + csa::topk_hist_bytes(p->B * T) : nullptr;
-  return launched(csa::launch_topk_select(*p, scores, ld, n_max, hist, q_pos0, T, out_idx, cand, st));
+  return launched(csa::launch_topk_select(*p, scores, p->score_fmt == CSA_SCORE_BF16, ld, n_max, hist, extra,
+                                          q_pos0, T, out_idx, st));
 }
 
 size_t csa_sparse_attn_workspace_bytes(const csa_params* p, int32_t T) {

@@ -397,11 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       S.row_lc[wt] = log2f(cj);
       S.row_ic[wt] = 1.f / cj;
     }
+    // Pair k of this warp: chunk group k % 9 (compile-time: groups 0-6 are
+    // E4M3 codes, 7-8 RoPE dims) of 8-row block warp + 8 (k / 9).
     uint4 raw[kLoads];
 #pragma unroll
     for (int k = 0; k < kLoads; ++k) {
-      const int pr = warp + 8 * k;
-      const int r = 8 * (pr / 9) + (lane >> 2), c = 4 * (pr % 9) + (lane & 3);
+      const int r = 8 * (warp + 8 * (k / 9)) + (lane >> 2), c = 4 * (k % 9) + (lane & 3);
       raw[k] = *reinterpret_cast<const uint4*>(stg + r * kRowBytes + c * 16);
     }
     __syncthreads();  // staging area read by all; row factors, live flags, query amax visible
@@ -426,10 +427,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     //    area holds stale bytes there)
 #pragma unroll
     for (int k = 0; k < kLoads; ++k) {
-      const int pr = warp + 8 * k;
-      const int r = 8 * (pr / 9) + (lane >> 2), c = 4 * (pr % 9) + (lane & 3);
+      const int r = 8 * (warp + 8 * (k / 9)) + (lane >> 2), c = 4 * (k % 9) + (lane & 3);
       const bool live = S.live[r] != 0;
-      if (c < kNope / 16) {
+      if (k % 9 < kNope / 64) {
         // dims 16c .. 16c+15 -> K-chunk (16c)/64, 16-byte slots 2(c%4), 2(c%4)+1;
         // codes times 2^k (exact down to 2^-24)
         uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;

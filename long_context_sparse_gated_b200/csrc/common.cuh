@@ -151,9 +151,18 @@ __device__ __forceinline__ uint32_t mxfp4_encode_quad(const float v[4], unsigned
   return (b0 & 0xFFu) | ((b1 & 0xFFu) << 8);
 }
 
-// Bins of the per-query score histogram: the top 12 bits of the key.
+// Order-preserving 16-bit key of a BF16 score (its bit pattern), -0 == +0.
+__device__ __forceinline__ uint32_t score_key16(uint32_t bits) {
+  bits &= 0xFFFFu;
+  if ((bits & 0x7FFFu) == 0) bits = 0;
+  return (bits & 0x8000u) ? (~bits & 0xFFFFu) : (bits | 0x8000u);
+}
+
+// Bins of the per-query score histogram: the top 12 bits of the key (of
+// the 32-bit key of an fp32 score, or of the 16-bit key of a BF16 score).
 constexpr int kScoreHistBins = 4096;
 __device__ __forceinline__ uint32_t score_bin(float f) { return score_key(f) >> 20; }
+__device__ __forceinline__ uint32_t score_bin16(uint32_t bits) { return score_key16(bits) >> 4; }
 
 // RoPE angle of pair j (of r/2) at position pos, in double precision so that
 // positions up to 2^20 and beyond keep a small absolute angle error.

@@ -21,7 +21,7 @@ template <int kHMax, int kC, bool kMx>
 __global__ void __launch_bounds__(256) index_scores_simt(
     const csa_params p, const void* __restrict__ q_idx, const uint8_t* __restrict__ q_sf,
     const float* __restrict__ w, const void* __restrict__ k_idx, const uint8_t* __restrict__ k_sf,
-    int64_t k_cap, const int32_t* __restrict__ q_pos0, int T, float* __restrict__ scores,
+    int64_t k_cap, const int32_t* __restrict__ q_pos0, int T, void* __restrict__ scores,
     int ld, int n_max, int32_t* __restrict__ err) {
   __shared__ float qs[kHMax * kC];
   __shared__ float ws[kHMax];
@@ -90,12 +90,15 @@ __global__ void __launch_bounds__(256) index_scores_simt(
 #pragma unroll
   for (int h = 0; h < kHMax; ++h)
     if (h < H) score = fmaf(ws[h], fmaxf(acc[h], 0.f), score);
-  scores[(int64_t)qi * ld + s] = score;
+  if (p.score_fmt == CSA_SCORE_BF16)
+    reinterpret_cast<uint16_t*>(scores)[(int64_t)qi * ld + s] = f32_to_bf16_bits(score);
+  else
+    reinterpret_cast<float*>(scores)[(int64_t)qi * ld + s] = score;
 }
 
 cudaError_t launch_index_scores(const csa_params& p, const void* q_idx, const uint8_t* q_sf,
                                 const float* w, const void* k_idx, const uint8_t* k_sf,
-                                int64_t k_cap, const int32_t* q_pos0, int T, float* scores,
+                                int64_t k_cap, const int32_t* q_pos0, int T, void* scores,
                                 int ld, int n_max, int32_t* err, cudaStream_t st) {
   dim3 grid(p.B * T, (n_max + 255) / 256);
   const bool mx = p.idx_fmt == CSA_IDX_MXFP4;

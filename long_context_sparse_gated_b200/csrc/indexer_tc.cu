@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     const __grid_constant__ CUtensorMap tm_key, const __grid_constant__ CUtensorMap tm_q,
     const __grid_constant__ CUtensorMap tm_sfk, const __grid_constant__ CUtensorMap tm_sfq,
     const float* __restrict__ w, const int32_t* __restrict__ q_pos0, int T, int m, int64_t k_cap,
-    int n_queries, int n_max, float* __restrict__ scores, int ld, uint32_t* __restrict__ hist,
+    int n_queries, int n_max, void* __restrict__ scores, int ld, int b16, uint32_t* __restrict__ hist,
     int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -345,8 +345,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       const float sc = (p4[0] + p4[1]) + (p4[2] + p4[3]);
       const int s_idx = j * kStageKeys + eg * kTileM + key_in_tile;
       if (s_idx < n_t) {
-        scores[(int64_t)qi * ld + s_idx] = sc;
-        if (hist) atomicAdd(sh + score_bin(sc), 1u);
+        // fp32 score, or rounded to BF16 (nearest even) for the BF16
+        // selector; the histogram bins the key the selector will rank
+        if (b16) {
+          const uint32_t bits = f32_to_bf16_bits(sc);
+          reinterpret_cast<uint16_t*>(scores)[(int64_t)qi * ld + s_idx] = (uint16_t)bits;
+          if (hist) atomicAdd(sh + score_bin16(bits), 1u);
+        } else {
+          reinterpret_cast<float*>(scores)[(int64_t)qi * ld + s_idx] = sc;
+          if (hist) atomicAdd(sh + score_bin(sc), 1u);
+        }
       }
     }
     if (hist && wq >= 0) flush(wq);
@@ -402,7 +410,7 @@ bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q
 
 cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const uint8_t* q_sf, const float* w,
                                    const void* k_idx, const uint8_t* k_sf, int64_t k_cap,
-                                   const int32_t* q_pos0, int T, float* scores, int ld, uint32_t* hist,
+                                   const int32_t* q_pos0, int T, void* scores, int ld, uint32_t* hist,
                                    int n_max, int32_t* err, cudaStream_t st) {
   const int nq = p.B * T;
   CUtensorMap tk, tq, tsk, tsq;
@@ -448,7 +456,7 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
   cudaError_t e = cudaFuncSetAttribute(index_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(index_scores_tc, dim3(grid), dim3(kThreadsTc), smem, st, tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap,
-                 nq, n_max, scores, ld, hist, err);
+                 nq, n_max, scores, ld, p.score_fmt == CSA_SCORE_BF16 ? 1 : 0, hist, err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

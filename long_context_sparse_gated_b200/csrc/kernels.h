@@ -57,9 +57,11 @@ cudaError_t launch_state_append(const csa_params& p, const void* kv_new, const v
 cudaError_t launch_state_restore(const csa_params& p, const int32_t* pos, const csa_ckpt& ck, const csa_state& s,
                                  int32_t* err, cudaStream_t st);
 
+// Scores are fp32, or BF16 (round to nearest even) when p.score_fmt is
+// CSA_SCORE_BF16; `scores` points to [B*T][ld] of either.
 cudaError_t launch_index_scores(const csa_params& p, const void* q_idx, const uint8_t* q_sf,
                                 const float* w, const void* k_idx, const uint8_t* k_sf,
-                                int64_t k_cap, const int32_t* q_pos0, int T, float* scores,
+                                int64_t k_cap, const int32_t* q_pos0, int T, void* scores,
                                 int ld, int n_max, int32_t* err, cudaStream_t st);
 
 bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q_idx, const uint8_t* q_sf,
@@ -67,16 +69,16 @@ bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q
 
 cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const uint8_t* q_sf, const float* w,
                                    const void* k_idx, const uint8_t* k_sf, int64_t k_cap,
-                                   const int32_t* q_pos0, int T, float* scores, int ld, uint32_t* hist,
+                                   const int32_t* q_pos0, int T, void* scores, int ld, uint32_t* hist,
                                    int n_max, int32_t* err, cudaStream_t st);
 
-size_t topk_hist_bytes(int queries);
 bool topk_use_hist(int queries);
 int topk_scores_ld(int n_max);
-size_t topk_cand_bytes(int queries, int n_max);
-cudaError_t launch_topk_select(const csa_params& p, const float* scores, int ld, int n_max,
-                               const uint32_t* hist, const int32_t* q_pos0, int T, int32_t* out_idx,
-                               void* cand, cudaStream_t st);
+size_t topk_zero_bytes(int queries);
+size_t topk_extra_bytes(int queries, int n_max);
+cudaError_t launch_topk_select(const csa_params& p, const void* scores, bool bf16, int ld, int n_max,
+                               const uint32_t* hist, void* extra, const int32_t* q_pos0, int T, int32_t* out_idx,
+                               cudaStream_t st);
 
 size_t attn_workspace_bytes(const csa_params& p, int T, int n_sel, bool dense);
 

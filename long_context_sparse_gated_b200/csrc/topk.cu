@@ -3,28 +3,37 @@
 // Qiaomu blog 混合注意力机制 and PACMAN notes 3.1: the selector keeps the
 // index_topk (512 for V4-Flash, 1024 for V4-Pro) highest-scoring compressed
 // entries of each query; ties go to the lower entry index, and the output
-// lists the entries in ascending order, padded with -1.
+// lists the entries in ascending order, padded with -1.  kwkr.cn notes 4.4:
+// the scores may be rounded from FP32 to BF16 before the selector (BF16
+// scores select on 16-bit keys).
 //
-// Scores become order-preserving 32-bit keys (larger score -> larger key,
-// -0 == +0).  One CTA (1024 threads) per query:
+// Scores become order-preserving keys (larger score -> larger key, -0 ==
+// +0): 32-bit for fp32 scores, 16-bit for BF16 scores.
 //
-//   1. threshold bin (histogram mode): the scoring kernel has counted every
-//      key's top 12 bits into a 4096-bin per-query histogram; a reverse scan
-//      finds the bin b* that holds the k-th largest key.  Without a
-//      histogram every entry is a candidate.
-//   2. one ordered pass over the scores copies every candidate (bin >= b*)
-//      into shared memory as (index, key), in ascending index order; each
-//      thread owns a contiguous run of 32 entries and one block-wide scan
-//      places the runs.
-//   3. an 8-bit radix select over the candidates' keys (warp-aggregated
-//      shared-memory histograms; 3 passes over the low 20 bits when the
-//      histogram fixed the top 12, else 4) finds the k-th largest key thr
-//      and how many entries equal to thr are taken (the lowest indices).
-//   4. an ordered compaction of the candidates (one contiguous run per
-//      thread, two block scans) writes the k entries, already ascending.
-// When the candidates do not fit in shared memory (heavy ties across a
-// huge range), the CTA falls back to the same radix select read from global
-// memory, then the same ordered compaction over all entries.
+// Histogram mode (the tensor-core scorer has counted every key's top 12
+// bits into a 4096-bin per-query histogram):
+//   1. threshold bin: a reverse scan of the histogram finds the bin b* that
+//      holds the k-th largest key, how many keys lie above it (cgt, all
+//      selected) and how many in it (nb, the ties of the first level);
+//   2. one pass over the scores: every entry above b* sets its bit in a
+//      selection bitmap; every entry in b* goes to a tie list and into a
+//      second-level histogram of its next 8 key bits (the last 4 for BF16);
+//   3. the second-level bin b2 holding the (k - cgt)-th tie: ties above it
+//      are selected, ties in it (a handful, or exact duplicates) are ranked
+//      by (key descending, index ascending) against each other;
+//   4. one block scan over the bitmap's popcounts writes the selected
+//      indices in ascending order.
+// Rows of up to 32768 entries run as one CTA per query (topk_fused); longer
+// rows run steps 1-2 as one CTA per 32768-entry chunk (topk_chunk_pass,
+// bitmap and tie list in the workspace) and steps 1, 3, 4 as one CTA per
+// query (topk_chunk_finish).  When the threshold bin holds more than
+// kTieCap entries (heavy ties), the query falls back to a radix select read
+// from global memory and an ordered compaction.
+//
+// Without a histogram (the CUDA-core scorer, or more than 4096 queries in
+// a call), every entry of a row of up to kCap entries is staged in shared
+// memory, a radix select finds the k-th key and an ordered compaction
+// writes the output; longer rows use the global-memory fallback.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -34,8 +43,59 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kPerThread = 32;
-constexpr int kChunk = kThreads * kPerThread;  // 32768 entries per ordered pass
-constexpr int kCap = 12288;                     // shared-memory candidates
+constexpr int kChunk = kThreads * kPerThread;  // 32768 entries per CTA pass
+constexpr int kCap = 12288;                     // staged keys (no-histogram mode)
+constexpr int kTieCap = 4096;                   // threshold-bin entries kept for steps 2-3
+constexpr int kSub = 256;                       // second-level bins
+
+// Keys of a score row: fp32 scores give 32-bit keys, BF16 scores 16-bit.
+template <bool kB16>
+struct ScoreKeys;
+
+template <>
+struct ScoreKeys<false> {
+  static constexpr int kBits = 32;
+  __device__ __forceinline__ static uint32_t key(const void* row, int s) {
+    return score_key(reinterpret_cast<const float*>(row)[s]);
+  }
+  // 32 consecutive keys from entry s0 (a multiple of 32)
+  __device__ __forceinline__ static void load32(const void* row, int s0, uint32_t (&k)[32]) {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row) + s0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 v = p[i];
+      k[4 * i] = score_key(v.x);
+      k[4 * i + 1] = score_key(v.y);
+      k[4 * i + 2] = score_key(v.z);
+      k[4 * i + 3] = score_key(v.w);
+    }
+  }
+  __device__ __forceinline__ static uint32_t bin(uint32_t key) { return key >> 20; }
+  __device__ __forceinline__ static uint32_t sub(uint32_t key) { return (key >> 12) & 0xFFu; }
+};
+
+template <>
+struct ScoreKeys<true> {
+  static constexpr int kBits = 16;
+  __device__ __forceinline__ static uint32_t key(const void* row, int s) {
+    return score_key16(reinterpret_cast<const uint16_t*>(row)[s]);
+  }
+  __device__ __forceinline__ static void load32(const void* row, int s0, uint32_t (&k)[32]) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(row) + s0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = p[i];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        k[8 * i + 2 * j] = score_key16(w[j]);
+        k[8 * i + 2 * j + 1] = score_key16(w[j] >> 16);
+      }
+    }
+  }
+  __device__ __forceinline__ static uint32_t bin(uint32_t key) { return key >> 4; }
+  __device__ __forceinline__ static uint32_t sub(uint32_t key) { return key & 0xFu; }
+};
 
 // exclusive scan of one int per thread over the 1024-thread block; returns
 // the prefix and writes the total to *total.  `tmp` holds >= 33 ints.
@@ -67,50 +127,43 @@ __device__ __forceinline__ int block_scan_excl(int v, int* tmp, int* total) {
   return r;
 }
 
-// exclusive scan of one uint64 per thread (four 16-bit counters packed, no
-// carries between them) over the 1024-thread block.  `tmp` holds >= 33
-// uint64.
-__device__ __forceinline__ uint64_t block_scan_excl64(uint64_t v, uint64_t* tmp, uint64_t* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  uint64_t incl = v;
+// In a 256-bin histogram h, the bin holding the `need`-th largest key
+// (1 <= need <= total count) and the count in higher bins, written to
+// out[0], out[1] by the one lane that finds them.  Warp 0 only.
+__device__ __forceinline__ void find_bin256(const uint32_t* h, uint32_t need, uint32_t* out) {
+  const int lane = threadIdx.x;
+  uint32_t c[8], tot = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { c[i] = h[255 - 8 * lane - i]; tot += c[i]; }
+  uint32_t incl = tot;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint64_t n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
-  if (lane == 31) tmp[wid] = incl;
-  __syncthreads();
-  if (wid == 0) {
-    const uint64_t w = tmp[lane];
-    uint64_t wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint64_t n = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += n;
+  const uint32_t before = incl - tot;
+  if (before < need && incl >= need) {
+    uint32_t acc = before;
+    for (int i = 0; i < 8; ++i) {
+      if (acc + c[i] >= need) {
+        out[0] = 255 - 8 * lane - i;
+        out[1] = acc;
+        break;
+      }
+      acc += c[i];
     }
-    tmp[lane] = wi - w;
-    if (lane == 31) tmp[32] = wi;
   }
-  __syncthreads();
-  const uint64_t r = tmp[wid] + incl - v;
-  *total = tmp[32];
-  __syncthreads();
-  return r;
 }
 
-// Radix select over n keys held by `get(i)` whose bits above `top_bit` all
-// equal those of `prefix0` (mask0 marks the known bits): the key of the
-// k-th largest (1 <= k <= n) and how many keys equal to it are among the
-// top k.  Passes take 8 bits, the last one the remainder.
-template <class Get>
-__device__ void radix_select(int n, int k, Get get, uint32_t prefix0, uint32_t mask0, int top_bit,
-                             uint32_t* hist, uint32_t* sel, uint32_t* thr_out, int* need_out) {
-  uint32_t prefix = prefix0, mask = mask0;
+// Radix select over n keys held by `get(i)` (the top `kBits` bits): the
+// key of the k-th largest (1 <= k <= n) and how many keys equal to it are
+// among the top k.  Passes take 8 bits.
+template <int kBits, class Get>
+__device__ void radix_select(int n, int k, Get get, uint32_t* hist, uint32_t* sel, uint32_t* thr_out,
+                             int* need_out) {
+  uint32_t prefix = 0, mask = 0;
   int remaining = k;
-  for (int hi = top_bit; hi >= 0; hi -= 8) {
-    const int width = hi >= 7 ? 8 : hi + 1;
-    const int shift = hi + 1 - width;
-    const uint32_t dmask = (1u << width) - 1u;
+  for (int shift = kBits - 8; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
     __syncthreads();
     for (int i0 = 0; i0 < n; i0 += kThreads) {
@@ -121,49 +174,34 @@ __device__ void radix_select(int n, int k, Get get, uint32_t prefix0, uint32_t m
         key = get(i);
         act = (key & mask) == prefix;
       }
-      hist_add(hist, (key >> shift) & dmask, act);
+      hist_add(hist, (key >> shift) & 0xFFu, act);
     }
     __syncthreads();
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      uint32_t c[8], tot = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { c[i] = hist[255 - 8 * lane - i]; tot += c[i]; }
-      uint32_t incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const uint32_t before = incl - tot;
-      if (before < (uint32_t)remaining && incl >= (uint32_t)remaining) {
-        uint32_t acc = before;
-        for (int i = 0; i < 8; ++i) {
-          if (acc + c[i] >= (uint32_t)remaining) {
-            sel[0] = 255 - 8 * lane - i;
-            sel[1] = acc;
-            break;
-          }
-          acc += c[i];
-        }
-      }
-    }
+    if (threadIdx.x < 32) find_bin256(hist, (uint32_t)remaining, sel);
     __syncthreads();
-    prefix |= sel[0] << shift;
-    mask |= dmask << shift;
-    remaining -= (int)sel[1];
+    const uint32_t bsel = sel[0], asel = sel[1];
+    __syncthreads();
+    prefix |= bsel << shift;
+    mask |= 0xFFu << shift;
+    remaining -= (int)asel;
   }
   *thr_out = prefix;
   *need_out = remaining;
 }
 
-struct TopkSmem;
-
 // The bin b* holding the k-th largest key, the count of entries in higher
-// bins (all selected) and of entries in bins >= b* (the candidates), from a
-// 4096-bin histogram of the keys' top 12 bits.  All threads must call.
+// bins (all selected) and in bins >= b*, from a 4096-bin histogram of the
+// keys' top 12 bits.  All threads must call.  *bstar < 0 when the
+// histogram holds fewer than k keys (it then does not describe the scores,
+// e.g. after the scorer gave up on a timed-out wait): callers fall back to
+// the global-memory selection, which reads only the scores.
 template <class Sm>
 __device__ void threshold_bin(const uint32_t* h, int k, Sm& S, int* bstar, int* cgt, int* ncand) {
+  if (threadIdx.x == 0) {
+    S.bstar = -1;
+    S.cgt = 0;
+    S.ncand = 0;
+  }
   // thread t owns bins 4095-4t .. 4092-4t (descending)
   uint32_t c[4], tot = 0;
 #pragma unroll
@@ -189,158 +227,30 @@ __device__ void threshold_bin(const uint32_t* h, int k, Sm& S, int* bstar, int* 
   __syncthreads();
 }
 
-// Ordered collection of one 32768-entry chunk [base, base+32768) of a score
-// row: every entry whose key's top 12 bits are >= bstar is appended, in
-// index order, as (index, key) to cidx/ckey.  Loads are coalesced: load i
-// (of 8) of thread t covers entries base + 4t + 4096 i .. +3; each thread's
-// 8 candidate counts are packed into two uint64 (four 16-bit fields each),
-// so two block scans give every load its position.  Returns the count.
-template <class Sm>
-__device__ int collect_chunk(const float* sc, int n_t, int base, int bstar, Sm& S, int* cidx, uint32_t* ckey) {
-  uint32_t keys[8][4];
-  uint64_t c01 = 0, c23 = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int s0 = base + 4 * threadIdx.x + 4096 * i;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (s0 < n_t) v = *reinterpret_cast<const float4*>(sc + s0);
-    const float f[4] = {v.x, v.y, v.z, v.w};
-    uint64_t cnt = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t key = score_key(f[e]);
-      const bool ok = (s0 + e < n_t) && (int)(key >> 20) >= bstar;
-      keys[i][e] = ok ? key : 0u;  // 0 marks a non-candidate (only -NaN maps to 0)
-      cnt += ok;
-    }
-    if (i < 4) c01 |= cnt << (16 * i);
-    else c23 |= cnt << (16 * (i - 4));
-  }
-  uint64_t t01, t23;
-  const uint64_t p01 = block_scan_excl64(c01, S.tmp64, &t01);
-  const uint64_t p23 = block_scan_excl64(c23, S.tmp64, &t23);
-  int lbase = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint64_t pf = i < 4 ? p01 : p23, tf = i < 4 ? t01 : t23;
-    const int sh = 16 * (i & 3);
-    int pos = lbase + (int)((pf >> sh) & 0xFFFFu);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (keys[i][e]) {
-        cidx[pos] = base + 4 * threadIdx.x + 4096 * i + e;
-        ckey[pos] = keys[i][e];
-        ++pos;
-      }
-    }
-    lbase += (int)((tf >> sh) & 0xFFFFu);
-  }
-  return lbase;
-}
-
-struct TopkSmem {
-  int cidx[kCap];
-  uint32_t ckey[kCap];
-  uint32_t hist[4096];
-  int tmp[40];
-  uint64_t tmp64[40];
+struct BitSmem {
+  uint32_t bits[kThreads];  // selection bitmap of a 32768-entry chunk
+  int tidx[kTieCap];        // threshold-bin entries: index and key
+  uint32_t tkey[kTieCap];
+  int grp[kTieCap];         // tie-list positions of the second-level bin b2
+  uint32_t h2[kSub];        // second-level histogram (also the fallback's radix histogram)
   uint32_t sel[2];
+  int tmp[40];
+  int tie_count, grp_count;
   int bstar, cgt, ncand;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) topk_select(const float* __restrict__ scores, int ld, int n_max,
-                                                            const uint32_t* __restrict__ ghist,
-                                                            const int32_t* __restrict__ q_pos0, int T, int m,
-                                                            int k, int32_t* __restrict__ out_idx,
-                                                            const int* __restrict__ cidx_g,
-                                                            const uint32_t* __restrict__ ckey_g,
-                                                            const int* __restrict__ ccount, int n_chunks) {
-  extern __shared__ uint8_t smem_raw[];
-  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
-  pdl_wait();
-  pdl_trigger();
-  const int qi = blockIdx.x;
-  const int bs = qi / T, tq = qi % T;
-  const int64_t t = (int64_t)q_pos0[bs] + tq;
-  int64_t n64 = (t + 1) / m;
-  if (n64 > n_max) n64 = n_max;
-  const int n_t = (int)n64;
-  const float* sc = scores + (int64_t)qi * ld;
-  int32_t* out = out_idx + (int64_t)qi * k;
-  if (n_t <= k) {
-    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n_t ? i : -1;
-    return;
-  }
-  // 1. threshold bin from the histogram (bins >= bstar are candidates)
-  int bstar = 0, cgt = 0, cand_total = n_t;
-  if (ghist) threshold_bin(ghist + (int64_t)qi * 4096, k, S, &bstar, &cgt, &cand_total);
-  bool fits = cand_total <= kCap;
-  if (fits && ccount && ccount[(int64_t)qi * n_chunks] < 0) fits = false;
-  if (fits) {
-    // 2. ordered candidate collection (or the chunk lists a collect pass
-    //    already wrote, concatenated in chunk order)
-    int base_out = 0;
-    if (ccount) {
-      for (int c = 0; c < n_chunks; ++c) {
-        const int cnt = ccount[(int64_t)qi * n_chunks + c];
-        const int64_t off = ((int64_t)qi * n_chunks + c) * kCap;
-        for (int i = threadIdx.x; i < cnt; i += kThreads) {
-          S.cidx[base_out + i] = cidx_g[off + i];
-          S.ckey[base_out + i] = ckey_g[off + i];
-        }
-        base_out += cnt;
-      }
-    } else {
-      for (int base = 0; base < n_t; base += kChunk)
-        base_out += collect_chunk(sc, n_t, base, bstar, S, S.cidx + base_out, S.ckey + base_out);
-    }
-    __syncthreads();
-    const int nc = base_out;
-    // 3. exact k-th largest: with a histogram the top 12 bits of the k-th
-    //    key are bstar, so only bits 19..0 remain (3 passes); without one,
-    //    all 32 bits (4 passes)
-    uint32_t thr;
-    int need;
-    if (ghist)
-      radix_select(nc, k - cgt, [&](int i) { return S.ckey[i]; }, (uint32_t)bstar << 20, 0xFFF00000u, 19, S.hist,
-                   S.sel, &thr, &need);
-    else
-      radix_select(nc, k, [&](int i) { return S.ckey[i]; }, 0u, 0u, 31, S.hist, S.sel, &thr, &need);
-    // keys above thr are all kept; keys == thr take `need` slots, lowest
-    // index first.  Every thread owns a contiguous run of candidates, so
-    // two block scans place the run's equal keys and its outputs in order.
-    const int per = (nc + kThreads - 1) / kThreads;
-    const int r0 = min(nc, threadIdx.x * per), r1 = min(nc, r0 + per);
-    int n_eq = 0;
-    for (int i = r0; i < r1; ++i) n_eq += S.ckey[i] == thr;
-    int tot;
-    int eq_rank = block_scan_excl(n_eq, S.tmp, &tot);
-    int n_sel = 0;
-    {
-      int er = eq_rank;
-      for (int i = r0; i < r1; ++i) {
-        const uint32_t key = S.ckey[i];
-        if (key > thr) ++n_sel;
-        else if (key == thr) n_sel += (er++ < need);
-      }
-    }
-    int pos = block_scan_excl(n_sel, S.tmp, &tot);
-    for (int i = r0; i < r1; ++i) {
-      const uint32_t key = S.ckey[i];
-      bool take = key > thr;
-      if (key == thr) take = eq_rank++ < need;
-      if (take) out[pos++] = S.cidx[i];
-    }
-    return;
-  }
-  // fallback: radix select straight from global memory
+// Global-memory fallback for a row (heavy ties): radix select over the
+// keys, then an ordered compaction, 1024 entries per step.
+template <bool kB16>
+__device__ void select_full(const void* row, int n_t, int k, int32_t* out, BitSmem& S) {
   uint32_t thr;
   int need;
-  radix_select(n_t, k, [&](int i) { return score_key(sc[i]); }, 0u, 0u, 31, S.hist, S.sel, &thr, &need);
+  radix_select<ScoreKeys<kB16>::kBits>(n_t, k, [&](int i) { return ScoreKeys<kB16>::key(row, i); }, S.h2, S.sel,
+                                       &thr, &need);
   int eq_base = 0, sel_base = 0;
   for (int i0 = 0; i0 < n_t; i0 += kThreads) {
     const int i = i0 + threadIdx.x;
-    const uint32_t key = i < n_t ? score_key(sc[i]) : 0u;
+    const uint32_t key = i < n_t ? ScoreKeys<kB16>::key(row, i) : 0u;
     const int eq = (i < n_t) && key == thr;
     int tot_eq, tot_sel;
     const int r_eq = eq_base + block_scan_excl(eq, S.tmp, &tot_eq);
@@ -352,90 +262,355 @@ __global__ void __launch_bounds__(kThreads, 1) topk_select(const float* __restri
   }
 }
 
-
-// Multi-CTA candidate pass for long score rows: CTA (query, chunk) appends
-// its chunk's candidates (bins >= b*) in index order to the chunk's slot of
-// the scratch lists; topk_select then concatenates the slots in order.
-__global__ void __launch_bounds__(kThreads, 1) topk_collect(const float* __restrict__ scores, int ld, int n_max,
-                                                             const uint32_t* __restrict__ ghist,
-                                                             const int32_t* __restrict__ q_pos0, int T, int m,
-                                                             int k, int* __restrict__ cidx_g,
-                                                             uint32_t* __restrict__ ckey_g, int* __restrict__ ccount,
-                                                             int n_chunks) {
-  extern __shared__ uint8_t smem_raw[];
-  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
-  pdl_wait();
-  pdl_trigger();
-  const int qi = blockIdx.x, chunk = blockIdx.y;
+__device__ __forceinline__ int visible_entries(const int32_t* q_pos0, int T, int m, int qi, int n_max) {
   const int bs = qi / T, tq = qi % T;
   const int64_t t = (int64_t)q_pos0[bs] + tq;
   int64_t n64 = (t + 1) / m;
   if (n64 > n_max) n64 = n_max;
-  const int n_t = (int)n64;
-  const int64_t slot = (int64_t)qi * n_chunks + chunk;
-  if (n_t <= k || chunk * kChunk >= n_t) {
-    if (threadIdx.x == 0) ccount[slot] = 0;
+  return (int)n64;
+}
+
+// Step 2 over this thread's 32 entries [s0, s0+32): its bitmap word (keys
+// above b*), and its threshold-bin entries appended to the tie list (warp-
+// aggregated slots from *count; slots past kTieCap are not written, and the
+// caller then falls back) and counted into the second-level histogram.
+// Every lane of the warp must call.
+template <bool kB16>
+__device__ __forceinline__ uint32_t scan32(const void* row, int s0, int n_t, int bstar, int* count, int* tidx,
+                                           uint32_t* tkey, uint32_t* h2) {
+  uint32_t keys[32];
+  uint32_t word = 0, tie = 0;
+  if (s0 < n_t) {
+    ScoreKeys<kB16>::load32(row, s0, keys);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const uint32_t b = ScoreKeys<kB16>::bin(keys[e]);
+      const bool in = s0 + e < n_t;
+      word |= (uint32_t)(in && b > (uint32_t)bstar) << e;
+      tie |= (uint32_t)(in && b == (uint32_t)bstar) << e;
+    }
+  }
+  const int lane = threadIdx.x & 31;
+  const int nt = __popc(tie);
+  int incl = nt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int base = 0;
+  if (lane == 31 && incl) base = atomicAdd(count, incl);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  int pos = base + incl - nt;
+  while (tie) {
+    const int e = __ffs(tie) - 1;
+    tie &= tie - 1;
+    if (pos < kTieCap) {
+      tidx[pos] = s0 + e;
+      tkey[pos] = keys[e];
+    }
+    atomicAdd(h2 + ScoreKeys<kB16>::sub(keys[e]), 1u);
+    ++pos;
+  }
+  return word;
+}
+
+// Steps 3: given the tie list in shared memory (S.tidx/S.tkey, nb entries)
+// and the second-level histogram, mark the ties that are selected via
+// mark(index).  `need` >= 1 ties are to be taken.
+template <bool kB16, class Mark>
+__device__ void resolve_ties(int nb, int need, BitSmem& S, Mark mark) {
+  if (threadIdx.x < 32) find_bin256(S.h2, (uint32_t)need, S.sel);
+  if (threadIdx.x == 0) S.grp_count = 0;
+  __syncthreads();
+  const uint32_t b2 = S.sel[0];
+  const int need2 = need - (int)S.sel[1];
+  for (int c = threadIdx.x; c < nb; c += kThreads) {
+    const uint32_t sb = ScoreKeys<kB16>::sub(S.tkey[c]);
+    if (sb > b2) mark(S.tidx[c]);
+    else if (sb == b2) S.grp[atomicAdd(&S.grp_count, 1)] = c;
+  }
+  __syncthreads();
+  const int n2 = S.grp_count;
+  for (int g = threadIdx.x; g < n2; g += kThreads) {
+    const int c = S.grp[g];
+    const uint32_t kc = S.tkey[c];
+    const int ic = S.tidx[c];
+    int rank = 0;
+    for (int h = 0; h < n2; ++h) {
+      const int c2 = S.grp[h];
+      const uint32_t k2 = S.tkey[c2];
+      rank += (k2 > kc) || (k2 == kc && S.tidx[c2] < ic);
+    }
+    if (rank < need2) mark(ic);
+  }
+  __syncthreads();
+}
+
+template <bool kB16>
+__device__ __forceinline__ const void* score_row(const void* scores, int64_t qi, int ld) {
+  return reinterpret_cast<const uint8_t*>(scores) + qi * ld * (kB16 ? 2 : 4);
+}
+
+// Histogram mode, rows of up to 32768 entries: one CTA per query.
+template <bool kB16>
+__global__ void __launch_bounds__(kThreads, 1) topk_fused(const void* __restrict__ scores, int ld, int n_max,
+                                                           const uint32_t* __restrict__ ghist,
+                                                           const int32_t* __restrict__ q_pos0, int T, int m, int k,
+                                                           int32_t* __restrict__ out_idx) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BitSmem& S = *reinterpret_cast<BitSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
+  const int qi = blockIdx.x;
+  const int n_t = visible_entries(q_pos0, T, m, qi, n_max);
+  const void* row = score_row<kB16>(scores, qi, ld);
+  int32_t* out = out_idx + (int64_t)qi * k;
+  if (n_t <= k) {
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n_t ? i : -1;
+    return;
+  }
+  if (threadIdx.x < kSub) S.h2[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) S.tie_count = 0;
+  int bstar, cgt, ncand;
+  threshold_bin(ghist + (int64_t)qi * kScoreHistBins, k, S, &bstar, &cgt, &ncand);
+  const int nb = ncand - cgt;
+  if (bstar < 0 || nb > kTieCap) {
+    select_full<kB16>(row, n_t, k, out, S);
+    return;
+  }
+  const int s0 = kPerThread * threadIdx.x;
+  S.bits[threadIdx.x] = scan32<kB16>(row, s0, n_t, bstar, &S.tie_count, S.tidx, S.tkey, S.h2);
+  __syncthreads();
+  if (S.tie_count != nb) {  // the histogram does not describe these scores
+    select_full<kB16>(row, n_t, k, out, S);
+    return;
+  }
+  resolve_ties<kB16>(nb, k - cgt, S, [&](int i) { atomicOr(&S.bits[i >> 5], 1u << (i & 31)); });
+  uint32_t word = S.bits[threadIdx.x];
+  int tot;
+  int pos = block_scan_excl(__popc(word), S.tmp, &tot);
+  while (word) {
+    const int e = __ffs(word) - 1;
+    word &= word - 1;
+    out[pos++] = s0 + e;
+  }
+}
+
+// Histogram mode, longer rows, step 1-2 per 32768-entry chunk: bitmap words
+// and tie list (with its count and second-level histogram) in the workspace.
+template <bool kB16>
+__global__ void __launch_bounds__(kThreads, 1) topk_chunk_pass(const void* __restrict__ scores, int ld, int n_max,
+                                                                const uint32_t* __restrict__ ghist,
+                                                                const int32_t* __restrict__ q_pos0, int T, int m,
+                                                                int k, uint32_t* __restrict__ gbits,
+                                                                int* __restrict__ gtidx, uint32_t* __restrict__ gtkey,
+                                                                int* __restrict__ gcount, uint32_t* __restrict__ gh2) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BitSmem& S = *reinterpret_cast<BitSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
+  const int qi = blockIdx.x, chunk = blockIdx.y;
+  const int n_t = visible_entries(q_pos0, T, m, qi, n_max);
+  const int base = chunk * kChunk;
+  if (n_t <= k || base >= n_t) return;
+  int bstar, cgt, ncand;
+  threshold_bin(ghist + (int64_t)qi * kScoreHistBins, k, S, &bstar, &cgt, &ncand);
+  if (bstar < 0 || ncand - cgt > kTieCap) return;  // topk_chunk_finish falls back
+  const int s0 = base + kPerThread * threadIdx.x;
+  const uint32_t word = scan32<kB16>(score_row<kB16>(scores, qi, ld), s0, n_t, bstar, gcount + qi,
+                                     gtidx + (int64_t)qi * kTieCap, gtkey + (int64_t)qi * kTieCap,
+                                     gh2 + (int64_t)qi * kSub);
+  if (s0 < n_t) gbits[(int64_t)qi * (ld / 32) + s0 / 32] = word;
+}
+
+// Histogram mode, longer rows, steps 3-4 per query.
+template <bool kB16>
+__global__ void __launch_bounds__(kThreads, 1) topk_chunk_finish(const void* __restrict__ scores, int ld, int n_max,
+                                                                  const uint32_t* __restrict__ ghist,
+                                                                  const int32_t* __restrict__ q_pos0, int T, int m,
+                                                                  int k, int32_t* __restrict__ out_idx,
+                                                                  uint32_t* __restrict__ gbits,
+                                                                  const int* __restrict__ gtidx,
+                                                                  const uint32_t* __restrict__ gtkey,
+                                                                  const int* __restrict__ gcount,
+                                                                  const uint32_t* __restrict__ gh2) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BitSmem& S = *reinterpret_cast<BitSmem*>(smem_raw);
+  pdl_wait();
+  pdl_trigger();
+  const int qi = blockIdx.x;
+  const int n_t = visible_entries(q_pos0, T, m, qi, n_max);
+  const void* row = score_row<kB16>(scores, qi, ld);
+  int32_t* out = out_idx + (int64_t)qi * k;
+  if (n_t <= k) {
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n_t ? i : -1;
     return;
   }
   int bstar, cgt, ncand;
-  threshold_bin(ghist + (int64_t)qi * 4096, k, S, &bstar, &cgt, &ncand);
-  if (ncand > kCap) {  // the selector falls back to a global radix select
-    if (threadIdx.x == 0) ccount[slot] = -1;
+  threshold_bin(ghist + (int64_t)qi * kScoreHistBins, k, S, &bstar, &cgt, &ncand);
+  const int nb = ncand - cgt;
+  if (bstar < 0 || nb > kTieCap || __ldcg(gcount + qi) != nb) {
+    select_full<kB16>(row, n_t, k, out, S);
     return;
   }
-  // chunk lists are collected in shared memory, then copied out
-  const int n = collect_chunk(scores + (int64_t)qi * ld, n_t, chunk * kChunk, bstar, S, S.cidx, S.ckey);
-  __syncthreads();
-  const int64_t off = slot * kCap;
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    cidx_g[off + i] = S.cidx[i];
-    ckey_g[off + i] = S.ckey[i];
+  if (threadIdx.x < kSub) S.h2[threadIdx.x] = __ldcg(gh2 + (int64_t)qi * kSub + threadIdx.x);
+  for (int c = threadIdx.x; c < nb; c += kThreads) {
+    S.tidx[c] = __ldcg(gtidx + (int64_t)qi * kTieCap + c);
+    S.tkey[c] = __ldcg(gtkey + (int64_t)qi * kTieCap + c);
   }
-  if (threadIdx.x == 0) ccount[slot] = n;
+  __syncthreads();
+  uint32_t* rowbits = gbits + (int64_t)qi * (ld / 32);
+  resolve_ties<kB16>(nb, k - cgt, S, [&](int i) { atomicOr(rowbits + (i >> 5), 1u << (i & 31)); });
+  // output: each thread owns a contiguous run of bitmap words
+  const int words = (n_t + 31) / 32;
+  const int per = (words + kThreads - 1) / kThreads;
+  const int w0 = min(words, (int)threadIdx.x * per), w1 = min(words, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(__ldcg(rowbits + w));
+  int tot;
+  int pos = block_scan_excl(cnt, S.tmp, &tot);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t word = __ldcg(rowbits + w);
+    while (word) {
+      const int e = __ffs(word) - 1;
+      word &= word - 1;
+      out[pos++] = 32 * w + e;
+    }
+  }
+}
+
+struct StageSmem {
+  uint32_t ckey[kCap];
+  uint32_t hist[256];
+  uint32_t sel[2];
+  int tmp[40];
+};
+
+// No-histogram mode: the whole row's keys staged in shared memory (rows up
+// to kCap entries), radix select, ordered compaction.
+template <bool kB16>
+__global__ void __launch_bounds__(kThreads, 1) topk_staged(const void* __restrict__ scores, int ld, int n_max,
+                                                            const int32_t* __restrict__ q_pos0, int T, int m, int k,
+                                                            int32_t* __restrict__ out_idx) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  pdl_wait();
+  pdl_trigger();
+  const int qi = blockIdx.x;
+  const int n_t = visible_entries(q_pos0, T, m, qi, n_max);
+  const void* row = score_row<kB16>(scores, qi, ld);
+  int32_t* out = out_idx + (int64_t)qi * k;
+  if (n_t <= k) {
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n_t ? i : -1;
+    return;
+  }
+  if (n_t > kCap) {
+    select_full<kB16>(row, n_t, k, out, *reinterpret_cast<BitSmem*>(smem_raw));
+    return;
+  }
+  StageSmem& S = *reinterpret_cast<StageSmem*>(smem_raw);
+  for (int s0 = kPerThread * threadIdx.x; s0 < n_t; s0 += kPerThread * kThreads) {
+    uint32_t keys[32];
+    ScoreKeys<kB16>::load32(row, s0, keys);
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (s0 + e < n_t) S.ckey[s0 + e] = keys[e];
+  }
+  __syncthreads();
+  uint32_t thr;
+  int need;
+  radix_select<ScoreKeys<kB16>::kBits>(n_t, k, [&](int i) { return S.ckey[i]; }, S.hist, S.sel, &thr, &need);
+  // keys above thr are all kept; keys == thr take `need` slots, lowest
+  // index first.  Every thread owns a contiguous run of entries, so two
+  // block scans place the run's equal keys and its outputs in order.
+  const int per = (n_t + kThreads - 1) / kThreads;
+  const int r0 = min(n_t, (int)threadIdx.x * per), r1 = min(n_t, r0 + per);
+  int n_eq = 0;
+  for (int i = r0; i < r1; ++i) n_eq += S.ckey[i] == thr;
+  int tot;
+  int eq_rank = block_scan_excl(n_eq, S.tmp, &tot);
+  int n_sel = 0;
+  {
+    int er = eq_rank;
+    for (int i = r0; i < r1; ++i) {
+      const uint32_t key = S.ckey[i];
+      if (key > thr) ++n_sel;
+      else if (key == thr) n_sel += (er++ < need);
+    }
+  }
+  int pos = block_scan_excl(n_sel, S.tmp, &tot);
+  for (int i = r0; i < r1; ++i) {
+    const uint32_t key = S.ckey[i];
+    bool take = key > thr;
+    if (key == thr) take = eq_rank++ < need;
+    if (take) out[pos++] = i;
+  }
+}
+
+template <class K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <bool kB16>
+cudaError_t launch_topk_t(const csa_params& p, const void* scores, int ld, int n_max, const uint32_t* hist,
+                          void* extra, const int32_t* q_pos0, int T, int32_t* out_idx, cudaStream_t st) {
+  const int nq = p.B * T;
+  cudaError_t e;
+  if (!hist) {
+    const size_t smem = sizeof(StageSmem) > sizeof(BitSmem) ? sizeof(StageSmem) : sizeof(BitSmem);
+    if ((e = set_smem(topk_staged<kB16>, smem)) != cudaSuccess) return e;
+    return launch_pdl(topk_staged<kB16>, dim3(nq), dim3(kThreads), smem, st, scores, ld, n_max, q_pos0, T, p.m,
+                      p.topk, out_idx);
+  }
+  const size_t smem = sizeof(BitSmem);
+  if (n_max <= kChunk) {
+    if ((e = set_smem(topk_fused<kB16>, smem)) != cudaSuccess) return e;
+    return launch_pdl(topk_fused<kB16>, dim3(nq), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T, p.m,
+                      p.topk, out_idx);
+  }
+  // the counters and second-level histograms follow the per-query
+  // histograms (cleared with them); bitmap and tie lists are in `extra`
+  int* gcount = reinterpret_cast<int*>(const_cast<uint32_t*>(hist) + (size_t)nq * kScoreHistBins);
+  uint32_t* gh2 = reinterpret_cast<uint32_t*>(gcount + ((nq + 3) & ~3));
+  uint32_t* gbits = reinterpret_cast<uint32_t*>(extra);
+  int* gtidx = reinterpret_cast<int*>(gbits + (size_t)nq * (ld / 32));
+  uint32_t* gtkey = reinterpret_cast<uint32_t*>(gtidx + (size_t)nq * kTieCap);
+  const int chunks = (n_max + kChunk - 1) / kChunk;
+  if ((e = set_smem(topk_chunk_pass<kB16>, smem)) != cudaSuccess) return e;
+  if ((e = set_smem(topk_chunk_finish<kB16>, smem)) != cudaSuccess) return e;
+  e = launch_pdl(topk_chunk_pass<kB16>, dim3(nq, chunks), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0,
+                 T, p.m, p.topk, gbits, gtidx, gtkey, gcount, gh2);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(topk_chunk_finish<kB16>, dim3(nq), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T,
+                    p.m, p.topk, out_idx, gbits, (const int*)gtidx, (const uint32_t*)gtkey, (const int*)gcount,
+                    (const uint32_t*)gh2);
 }
 
 }  // namespace
-
-size_t topk_hist_bytes(int queries) { return (size_t)queries * 4096 * sizeof(uint32_t); }
 
 bool topk_use_hist(int queries) { return queries <= 4096; }
 
 int topk_scores_ld(int n_max) { return (n_max + 31) & ~31; }
 
-// Chunked candidate lists for long rows (histogram mode, n_max > 32768):
-// [queries][chunks][kCap] indices and keys, then [queries][chunks] counts.
-int topk_chunks(int n_max) { return (n_max + kChunk - 1) / kChunk; }
-
-size_t topk_cand_bytes(int queries, int n_max) {
-  const int c = topk_chunks(n_max);
-  if (c <= 1) return 0;
-  return (size_t)queries * c * ((size_t)kCap * 8 + 4);
+// Cleared region of histogram mode: per-query 4096-bin histograms, tie
+// counts (padded to 16 bytes) and 256-bin second-level histograms.
+size_t topk_zero_bytes(int queries) {
+  return (size_t)queries * kScoreHistBins * 4 + (size_t)((queries + 3) & ~3) * 4 + (size_t)queries * kSub * 4;
 }
 
-cudaError_t launch_topk_select(const csa_params& p, const float* scores, int ld, int n_max,
-                               const uint32_t* hist, const int32_t* q_pos0, int T, int32_t* out_idx,
-                               void* cand, cudaStream_t st) {
-  const size_t smem = sizeof(TopkSmem);
-  const int nq = p.B * T;
-  const int chunks = topk_chunks(n_max);
-  int* cidx = nullptr;
-  uint32_t* ckey = nullptr;
-  int* ccount = nullptr;
-  if (hist && chunks > 1 && cand) {
-    cidx = reinterpret_cast<int*>(cand);
-    ckey = reinterpret_cast<uint32_t*>(cidx + (size_t)nq * chunks * kCap);
-    ccount = reinterpret_cast<int*>(ckey + (size_t)nq * chunks * kCap);
-    cudaError_t e = cudaFuncSetAttribute(topk_collect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(topk_collect, dim3(nq, chunks), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T,
-                   p.m, p.topk, cidx, ckey, ccount, chunks);
-    if (e != cudaSuccess) return e;
-  }
-  cudaError_t e = cudaFuncSetAttribute(topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(topk_select, dim3(nq), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T, p.m,
-                    p.topk, out_idx, (const int*)cidx, (const uint32_t*)ckey, (const int*)ccount,
-                    ccount ? chunks : 0);
+// Histogram mode with rows over 32768 entries: selection bitmaps and tie
+// lists.
+size_t topk_extra_bytes(int queries, int n_max) {
+  if (n_max <= kChunk) return 0;
+  return (size_t)queries * (topk_scores_ld(n_max) / 32) * 4 + (size_t)queries * kTieCap * 8;
+}
+
+cudaError_t launch_topk_select(const csa_params& p, const void* scores, bool bf16, int ld, int n_max,
+                               const uint32_t* hist, void* extra, const int32_t* q_pos0, int T, int32_t* out_idx,
+                               cudaStream_t st) {
+  return bf16 ? launch_topk_t<true>(p, scores, ld, n_max, hist, extra, q_pos0, T, out_idx, st)
+              : launch_topk_t<false>(p, scores, ld, n_max, hist, extra, q_pos0, T, out_idx, st);
 }
 
 }  // namespace csa

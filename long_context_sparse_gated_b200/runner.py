@@ -12,7 +12,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (ACT_BF16, ACT_F32, IDX_F32, IDX_MXFP4, KV_F32, KV_FP8_BF16, csa_compress,
+from . import (ACT_BF16, ACT_F32, IDX_F32, IDX_MXFP4, KV_F32, KV_FP8_BF16, SCORE_BF16, SCORE_F32, csa_compress,
                csa_index_topk, csa_index_topk_workspace_bytes, csa_sparse_attn,
                csa_sparse_attn_workspace_bytes, hca_compress, hca_dense_attn,
                hca_dense_attn_workspace_bytes, make_params)
@@ -31,7 +31,8 @@ def params_of(p):
     return make_params(B=p.B, d=p.d, r=p.r, m=p.m, n_idx_heads=p.H_I, idx_dim=p.c_I,
                        topk=max(p.k, 1), n_heads=p.n_h, window=p.W, kv_fmt=_KV[p.kv_fmt],
                        idx_fmt=_IDX[p.idx_fmt], act_fmt=_ACT[p.act_fmt], softmax_scale=p.tau,
-                       rope_theta=p.theta, eps=p.eps)
+                       rope_theta=p.theta, eps=p.eps,
+                       score_fmt=SCORE_BF16 if getattr(p, "score_fmt", "f32") == "bf16" else SCORE_F32)
 
 
 def _t(x, device):

@@ -64,6 +64,7 @@ class Params:
     kv_fmt: str = FMT_FP8
     idx_fmt: str = FMT_MXFP4
     act_fmt: str = FMT_BF16
+    score_fmt: str = "f32"   # index-score precision the selector ranks ("f32" or "bf16")
 
     @property
     def row_bytes(self) -> int:
@@ -362,6 +363,26 @@ def with_heads(w, n_h: int):
     w["params"] = dataclasses.replace(p, n_h=n_h)
     w["q"] = np.ascontiguousarray(w["q"][:, :, :n_h])
     w["sink"] = np.ascontiguousarray(w["sink"][:n_h])
+    return w
+
+
+def with_score_fmt(w, fmt: str):
+    """The workload with index scores ranked in ``fmt`` ("f32" or "bf16")."""
+    w = dict(w)
+    w["params"] = dataclasses.replace(w["params"], score_fmt=fmt)
+    return w
+
+
+def with_index_heads(w, n: int):
+    """The workload with only its first ``n`` index heads (index queries,
+    their scales and head weights sliced)."""
+    p = w["params"]
+    assert n <= p.H_I
+    w = dict(w)
+    w["params"] = dataclasses.replace(p, H_I=n)
+    for k in ("q_idx", "q_idx_sf", "w_idx"):
+        if k in w and w[k] is not None:
+            w[k] = np.ascontiguousarray(w[k][:, :, :n])
     return w
 
 

@@ -14,6 +14,12 @@ import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
+# csa_index_topk workspace for 2 queries over 32768 entries (fp32 scores):
+# the scores, then the cleared region (per query a 4096-bin histogram, a tie
+# count padded to 16 bytes over the batch, a 256-bin second-level
+# histogram), each rounded up to 256 bytes
+_INDEX_WS_2x32768 = 2 * 32768 * 4 + ((2 * 4096 * 4 + 16 + 2 * 256 * 4 + 255) // 256) * 256
+
 
 def _declared():
     src = open(os.path.join(ROOT, "include", "csa.h")).read()
@@ -89,7 +95,7 @@ def test_host_validation_codes():
     assert r["restore_null"] == -1
     assert r["quant_dim"] == -2
     assert r["ikc_rope"] == -2
-    assert r["ws_bytes"] == 2 * 32768 * 4 + 2 * 4096 * 4  # scores + per-query histograms
+    assert r["ws_bytes"] == _INDEX_WS_2x32768
     assert r["attn_ws"] > 0
     assert r["name"] == "CSA_ERR_WORKSPACE"
 
@@ -113,5 +119,5 @@ def test_plain_c_client_compiles_links_and_validates(tmp_path):
     assert out.returncode == 0, out.stderr
     s_null, s_bad, s_align, ws, name = out.stdout.split()
     assert (int(s_null), int(s_bad), int(s_align)) == (-1, -2, -3)
-    assert int(ws) == 2 * 32768 * 4 + 2 * 4096 * 4
+    assert int(ws) == _INDEX_WS_2x32768
     assert name == "CSA_ERR_ALIGN"

@@ -2,11 +2,10 @@
 
 On MXFP4 workloads whose scores are exactly representable in fp32 (the
 workload generator checks the bound), the fp32 scores the indexer writes to
-its workspace must equal the oracle's exact fp64 scores bit for bit, and the
-CUDA-core indexer (CSA_INDEXER=simt) must produce the same bits.
+its workspace must equal the oracle's exact fp64 scores bit for bit; so must
+the CUDA-core indexer, which serves the shapes the tensor-core one does not
+(here: 32 index heads).
 """
-
-import os
 
 import numpy as np
 import pytest
@@ -34,22 +33,11 @@ def _scores(dw):
     return dw.ws_idx.view(torch.float32)[:n].view(dw.p.B * dw.T, ld)[:, :dw.n_max].cpu().numpy()
 
 
-def _run_index(w, simt=False):
+def _run_index(w):
     from long_context_sparse_gated_b200.runner import DeviceWorkload
     dw = DeviceWorkload(w)
-    old = os.environ.get("CSA_INDEXER")
-    try:
-        if simt:
-            os.environ["CSA_INDEXER"] = "simt"
-        else:
-            os.environ.pop("CSA_INDEXER", None)
-        dw.index_topk()
-        torch.cuda.synchronize()
-    finally:
-        if old is None:
-            os.environ.pop("CSA_INDEXER", None)
-        else:
-            os.environ["CSA_INDEXER"] = old
+    dw.index_topk()
+    torch.cuda.synchronize()
     assert dw.err_bits() == 0
     return dw
 
@@ -73,11 +61,16 @@ def test_tc_scores_exact(name, kw):
         assert bad.size == 0, f"b={b}: {bad.size} inexact scores, first {bad[:5]} gpu {row[bad[:5]]} ref {sc[bad[:5]]}"
 
 
-def test_tc_matches_simt_bits():
-    w = synth.config("c1", B=2, L=8192)
-    a = _scores(_run_index(w))
-    b = _scores(_run_index(w, simt=True))
-    np.testing.assert_array_equal(a.view(np.uint32), b.view(np.uint32))
+def test_cuda_core_indexer_scores_and_topk_exact():
+    """32 index heads run on the CUDA-core scorer (no histogram: the staged
+    selector); scores and top-k sets equal the oracle's exactly."""
+    w = synth.with_index_heads(synth.config("c1", B=2, L=8192), 32)
+    dw = _run_index(w)
+    g = _scores(dw)
+    idx, scores = pipeline.index_topk(w, return_scores=True)
+    for (b, tq), sc in scores.items():
+        np.testing.assert_array_equal(g[b, :len(sc)].astype(np.float64), sc)
+        np.testing.assert_array_equal(dw.idx[b, tq].cpu().numpy(), idx[(b, tq)])
 
 
 def test_tc_prefill_many_queries():
