@@ -466,6 +466,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch every call from the host (no CUDA graphs)")
     ap.add_argument("--copies", type=int, default=0,
                     help="device copies rotated in the timed loop (0: enough to exceed 3x L2)")
+    ap.add_argument("--score-fmt", default="f32", choices=["f32", "bf16"],
+                    help="index-score precision the selector ranks (bf16: the BF16-score variant)")
     ap.add_argument("--extra-configs", default="c2,c3,c4",
                     help="with --config c1 on one GPU: the other workloads measured into the same line")
     args = ap.parse_args()
@@ -520,7 +522,7 @@ def run_config(config, args, world, rank, local):
     import torch.distributed as dist
     from long_context_sparse_gated_b200.runner import STEP_INPUTS, DeviceWorkload
 
-    w = synth.config(config, seed=rank_seed(config, rank))
+    w = synth.with_score_fmt(synth.config(config, seed=rank_seed(config, rank)), args.score_fmt)
     step_bytes, idx_bytes = algorithmic_bytes(w)
     n_copies = max(1, int(np.ceil(3 * L2_BYTES / step_bytes)))
     if config == "c4":
@@ -725,7 +727,7 @@ def run_config(config, args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8/bf16 storage, mxfp4 indexer, fp32 accumulate" if p.kv_fmt == "fp8" else "f32",
         "data": "synthetic",
-        "config": {"workload": CONFIG_NAMES[config], "name": config, "batch": p.B,
+        "config": {"workload": CONFIG_NAMES[config], "name": config, "batch": p.B, "index_scores": args.score_fmt,
                    "context": int(w["L"].max()), "queries_per_step": queries,
                    "l2": f"inputs larger than L2: {n_copies} device copies rotated, {n_copies * step_bytes / 2**20:.0f} MiB per cycle"},
         "gpu_launches": args.steps * (kernels_per_step if kernels_per_step is not None else launches_per_step(w)),

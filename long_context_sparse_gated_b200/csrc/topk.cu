@@ -15,12 +15,14 @@
 //   1. threshold bin: a reverse scan of the histogram finds the bin b* that
 //      holds the k-th largest key, how many keys lie above it (cgt, all
 //      selected) and how many in it (nb, the ties of the first level);
-//   2. one pass over the scores: every entry above b* sets its bit in a
-//      selection bitmap; every entry in b* goes to a tie list and into a
+//   2. one pass over the scores (coalesced 16-byte loads; warp ballots
+//      re-packed into 32-entry words): every entry above b* sets its bit in
+//      a selection bitmap; every entry in b* goes to a tie list and into a
 //      second-level histogram of its next 8 key bits (the last 4 for BF16);
 //   3. the second-level bin b2 holding the (k - cgt)-th tie: ties above it
-//      are selected, ties in it (a handful, or exact duplicates) are ranked
-//      by (key descending, index ascending) against each other;
+//      are selected; ties in it are ranked by (key descending, index
+//      ascending) -- pairwise for a handful, else by a radix select of the
+//      exact threshold key and an index bitmap of the keys equal to it;
 //   4. one block scan over the bitmap's popcounts writes the selected
 //      indices in ascending order.
 // Rows of up to 32768 entries run as one CTA per query (topk_fused); longer
@@ -47,6 +49,8 @@ constexpr int kChunk = kThreads * kPerThread;  // 32768 entries per CTA pass
 constexpr int kCap = 12288;                     // staged keys (no-histogram mode)
 constexpr int kTieCap = 4096;                   // threshold-bin entries kept for steps 2-3
 constexpr int kSub = 256;                       // second-level bins
+constexpr int kSmallGroup = 64;                 // final tie groups ranked pairwise up to this size
+constexpr int kEqWords = 8192;                  // index-bitmap window of equal keys (262144 entries)
 
 // Keys of a score row: fp32 scores give 32-bit keys, BF16 scores 16-bit.
 template <bool kB16>
@@ -58,18 +62,6 @@ struct ScoreKeys<false> {
   __device__ __forceinline__ static uint32_t key(const void* row, int s) {
     return score_key(reinterpret_cast<const float*>(row)[s]);
   }
-  // 32 consecutive keys from entry s0 (a multiple of 32)
-  __device__ __forceinline__ static void load32(const void* row, int s0, uint32_t (&k)[32]) {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row) + s0);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 v = p[i];
-      k[4 * i] = score_key(v.x);
-      k[4 * i + 1] = score_key(v.y);
-      k[4 * i + 2] = score_key(v.z);
-      k[4 * i + 3] = score_key(v.w);
-    }
-  }
   __device__ __forceinline__ static uint32_t bin(uint32_t key) { return key >> 20; }
   __device__ __forceinline__ static uint32_t sub(uint32_t key) { return (key >> 12) & 0xFFu; }
 };
@@ -79,19 +71,6 @@ struct ScoreKeys<true> {
   static constexpr int kBits = 16;
   __device__ __forceinline__ static uint32_t key(const void* row, int s) {
     return score_key16(reinterpret_cast<const uint16_t*>(row)[s]);
-  }
-  __device__ __forceinline__ static void load32(const void* row, int s0, uint32_t (&k)[32]) {
-    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(row) + s0);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = p[i];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        k[8 * i + 2 * j] = score_key16(w[j]);
-        k[8 * i + 2 * j + 1] = score_key16(w[j] >> 16);
-      }
-    }
   }
   __device__ __forceinline__ static uint32_t bin(uint32_t key) { return key >> 4; }
   __device__ __forceinline__ static uint32_t sub(uint32_t key) { return key & 0xFu; }
@@ -232,7 +211,8 @@ struct BitSmem {
   int tidx[kTieCap];        // threshold-bin entries: index and key
   uint32_t tkey[kTieCap];
   int grp[kTieCap];         // tie-list positions of the second-level bin b2
-  uint32_t h2[kSub];        // second-level histogram (also the fallback's radix histogram)
+  uint32_t eq[kEqWords];    // entries whose key equals the final threshold (by index), one window
+  uint32_t h2[kSub];        // second-level histogram (also the radix histogram)
   uint32_t sel[2];
   int tmp[40];
   int tie_count, grp_count;
@@ -270,27 +250,78 @@ __device__ __forceinline__ int visible_entries(const int32_t* q_pos0, int T, int
   return (int)n64;
 }
 
-// Step 2 over this thread's 32 entries [s0, s0+32): its bitmap word (keys
-// above b*), and its threshold-bin entries appended to the tie list (warp-
-// aggregated slots from *count; slots past kTieCap are not written, and the
-// caller then falls back) and counted into the second-level histogram.
-// Every lane of the warp must call.
+// Bit j of the low 8 bits of x moved to bit 4j (j < 8), and bit j of the
+// low 4 bits to bit 8j (j < 4).
+__device__ __forceinline__ uint32_t spread4(uint32_t x) {
+  x &= 0xFFu;
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x;
+}
+__device__ __forceinline__ uint32_t spread8(uint32_t x) {
+  x &= 0xFu;
+  x = (x | (x << 14)) & 0x00030003u;
+  x = (x | (x << 7)) & 0x01010101u;
+  return x;
+}
+
+// Step 2 over one 32768-entry chunk [base, base + 32768) of a score row, by
+// the whole CTA with coalesced 16-byte loads: fp32 rows in 8 passes of 4096
+// entries (lane l of warp w takes entries 4l..4l+3 of the warp's 128), BF16
+// rows in 4 passes of 8192 (8 entries per lane, 256 per warp).  Keys above
+// b* become bits of the selection bitmap: a warp's ballots, one per entry
+// slot of a lane, are re-packed into 32-entry words (words[j] for entries
+// base + 32j .. +31, written when j < n_words).  The threshold bin's
+// entries are appended to the tie list (warp-aggregated slots from *count;
+// slots past kTieCap are not written, and the caller then falls back) and
+// counted into the second-level histogram.
 template <bool kB16>
-__device__ __forceinline__ uint32_t scan32(const void* row, int s0, int n_t, int bstar, int* count, int* tidx,
-                                           uint32_t* tkey, uint32_t* h2) {
-  uint32_t keys[32];
-  uint32_t word = 0, tie = 0;
-  if (s0 < n_t) {
-    ScoreKeys<kB16>::load32(row, s0, keys);
+__device__ __forceinline__ void scan_chunk(const void* row, int base, int n_t, int bstar, uint32_t* words, int n_words,
+                                           int* count, int* tidx, uint32_t* tkey, uint32_t* h2) {
+  constexpr int kPer = kB16 ? 8 : 4;        // entries per lane per pass
+  constexpr int kPasses = 32 / kPer;        // passes per chunk
+  constexpr int kWarpSpan = 32 * kPer;      // entries per warp per pass
+  constexpr int kPassSpan = kThreads * kPer;
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  uint32_t tie = 0;  // bit kPer*i + e: entry (pass i, slot e) is in the threshold bin
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const uint32_t b = ScoreKeys<kB16>::bin(keys[e]);
-      const bool in = s0 + e < n_t;
-      word |= (uint32_t)(in && b > (uint32_t)bstar) << e;
-      tie |= (uint32_t)(in && b == (uint32_t)bstar) << e;
+  for (int i = 0; i < kPasses; ++i) {
+    const int s = base + kPassSpan * i + kWarpSpan * wp + kPer * lane;
+    uint32_t k[kPer];
+    if (s < n_t) {
+      if (kB16) {
+        const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(row) + s);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          k[2 * j] = score_key16(w[j]);
+          k[2 * j + 1] = score_key16(w[j] >> 16);
+        }
+      } else {
+        const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row) + s);
+        k[0] = score_key(v.x);
+        k[1] = score_key(v.y);
+        k[2] = score_key(v.z);
+        k[3] = score_key(v.w);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) k[e] = 0u;
     }
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const bool in = s + e < n_t;
+      const uint32_t b = ScoreKeys<kB16>::bin(k[e]);
+      tie |= (uint32_t)(in && b == (uint32_t)bstar) << (kPer * i + e);
+      const uint32_t m = __ballot_sync(0xffffffffu, in && b > (uint32_t)bstar);
+      // word q of this warp's span: lanes (32/kPer) q .. +32/kPer-1, slot e
+      word |= (kB16 ? spread8(m >> (4 * (lane & 7))) : spread4(m >> (8 * (lane & 3)))) << e;
+    }
+    const int j = (kPassSpan * i + kWarpSpan * wp) / 32 + lane;  // valid for lane < kPer
+    if (lane < kPer && j < n_words) words[j] = word;
   }
-  const int lane = threadIdx.x & 31;
   const int nt = __popc(tie);
   int incl = nt;
 #pragma unroll
@@ -298,28 +329,35 @@ __device__ __forceinline__ uint32_t scan32(const void* row, int s0, int n_t, int
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  int base = 0;
-  if (lane == 31 && incl) base = atomicAdd(count, incl);
-  base = __shfl_sync(0xffffffffu, base, 31);
-  int pos = base + incl - nt;
+  int pos = 0;
+  if (lane == 31 && incl) pos = atomicAdd(count, incl);
+  pos = __shfl_sync(0xffffffffu, pos, 31) + incl - nt;
   while (tie) {
-    const int e = __ffs(tie) - 1;
+    const int bit = __ffs(tie) - 1;
     tie &= tie - 1;
+    const int i = bit / kPer, e = bit % kPer;
+    const int idx = base + kPassSpan * i + kWarpSpan * wp + kPer * lane + e;
+    const uint32_t key = ScoreKeys<kB16>::key(row, idx);  // re-read: ties are few, the line is cached
     if (pos < kTieCap) {
-      tidx[pos] = s0 + e;
-      tkey[pos] = keys[e];
+      tidx[pos] = idx;
+      tkey[pos] = key;
     }
-    atomicAdd(h2 + ScoreKeys<kB16>::sub(keys[e]), 1u);
+    atomicAdd(h2 + ScoreKeys<kB16>::sub(key), 1u);
     ++pos;
   }
-  return word;
 }
 
-// Steps 3: given the tie list in shared memory (S.tidx/S.tkey, nb entries)
+// Step 3: given the tie list in shared memory (S.tidx/S.tkey, nb entries)
 // and the second-level histogram, mark the ties that are selected via
-// mark(index).  `need` >= 1 ties are to be taken.
+// mark(index).  `need` >= 1 ties are to be taken from a row of n_t entries.
+// The second-level bin b2 holding the need-th tie splits them: ties above
+// b2 are taken, ties in it form the final group.  A small group is ranked
+// pairwise by (key descending, index ascending).  A larger one (many equal
+// scores) gets a radix select of its exact threshold key; keys above it are
+// taken, and keys equal to it are flagged in an index bitmap whose prefix
+// popcounts rank them by index, lowest first.
 template <bool kB16, class Mark>
-__device__ void resolve_ties(int nb, int need, BitSmem& S, Mark mark) {
+__device__ void resolve_ties(int nb, int need, int n_t, BitSmem& S, Mark mark) {
   if (threadIdx.x < 32) find_bin256(S.h2, (uint32_t)need, S.sel);
   if (threadIdx.x == 0) S.grp_count = 0;
   __syncthreads();
@@ -332,17 +370,58 @@ __device__ void resolve_ties(int nb, int need, BitSmem& S, Mark mark) {
   }
   __syncthreads();
   const int n2 = S.grp_count;
-  for (int g = threadIdx.x; g < n2; g += kThreads) {
-    const int c = S.grp[g];
-    const uint32_t kc = S.tkey[c];
-    const int ic = S.tidx[c];
-    int rank = 0;
-    for (int h = 0; h < n2; ++h) {
-      const int c2 = S.grp[h];
-      const uint32_t k2 = S.tkey[c2];
-      rank += (k2 > kc) || (k2 == kc && S.tidx[c2] < ic);
+  if (n2 <= kSmallGroup) {
+    if ((int)threadIdx.x < n2) {
+      const int c = S.grp[threadIdx.x];
+      const uint32_t kc = S.tkey[c];
+      const int ic = S.tidx[c];
+      int rank = 0;
+      for (int h = 0; h < n2; ++h) {
+        const int c2 = S.grp[h];
+        const uint32_t k2 = S.tkey[c2];
+        rank += (k2 > kc) || (k2 == kc && S.tidx[c2] < ic);
+      }
+      if (rank < need2) mark(ic);
     }
-    if (rank < need2) mark(ic);
+    __syncthreads();
+    return;
+  }
+  uint32_t thr;
+  int need_eq;
+  radix_select<ScoreKeys<kB16>::kBits>(n2, need2, [&](int i) { return S.tkey[S.grp[i]]; }, S.h2, S.sel, &thr,
+                                       &need_eq);
+  for (int g = threadIdx.x; g < n2; g += kThreads)
+    if (S.tkey[S.grp[g]] > thr) mark(S.tidx[S.grp[g]]);
+  // equal keys: the need_eq lowest indices, window by window of the row
+  const int n_words = (n_t + 31) / 32;
+  int taken = 0;
+  for (int w0 = 0; w0 < n_words && taken < need_eq; w0 += kEqWords) {
+    for (int j = threadIdx.x; j < kEqWords; j += kThreads) S.eq[j] = 0u;
+    __syncthreads();
+    for (int g = threadIdx.x; g < n2; g += kThreads) {
+      const int c = S.grp[g];
+      const int w = (S.tidx[c] >> 5) - w0;
+      if (S.tkey[c] == thr && w >= 0 && w < kEqWords) atomicOr(&S.eq[w], 1u << (S.tidx[c] & 31));
+    }
+    __syncthreads();
+    constexpr int kPer = kEqWords / kThreads;  // words per thread, in index order
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) cnt += __popc(S.eq[kPer * threadIdx.x + j]);
+    int tot;
+    int rank = taken + block_scan_excl(cnt, S.tmp, &tot);
+#pragma unroll 1
+    for (int j = 0; j < kPer && rank < need_eq; ++j) {
+      uint32_t word = S.eq[kPer * threadIdx.x + j];
+      while (word && rank < need_eq) {
+        const int e = __ffs(word) - 1;
+        word &= word - 1;
+        mark(32 * (w0 + kPer * (int)threadIdx.x + j) + e);
+        ++rank;
+      }
+    }
+    taken += tot;
+    __syncthreads();
   }
   __syncthreads();
 }
@@ -379,21 +458,20 @@ __global__ void __launch_bounds__(kThreads, 1) topk_fused(const void* __restrict
     select_full<kB16>(row, n_t, k, out, S);
     return;
   }
-  const int s0 = kPerThread * threadIdx.x;
-  S.bits[threadIdx.x] = scan32<kB16>(row, s0, n_t, bstar, &S.tie_count, S.tidx, S.tkey, S.h2);
+  scan_chunk<kB16>(row, 0, n_t, bstar, S.bits, kThreads, &S.tie_count, S.tidx, S.tkey, S.h2);
   __syncthreads();
   if (S.tie_count != nb) {  // the histogram does not describe these scores
     select_full<kB16>(row, n_t, k, out, S);
     return;
   }
-  resolve_ties<kB16>(nb, k - cgt, S, [&](int i) { atomicOr(&S.bits[i >> 5], 1u << (i & 31)); });
+  resolve_ties<kB16>(nb, k - cgt, n_t, S, [&](int i) { atomicOr(&S.bits[i >> 5], 1u << (i & 31)); });
   uint32_t word = S.bits[threadIdx.x];
   int tot;
   int pos = block_scan_excl(__popc(word), S.tmp, &tot);
   while (word) {
     const int e = __ffs(word) - 1;
     word &= word - 1;
-    out[pos++] = s0 + e;
+    out[pos++] = kPerThread * threadIdx.x + e;
   }
 }
 
@@ -417,11 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1) topk_chunk_pass(const void* __res
   int bstar, cgt, ncand;
   threshold_bin(ghist + (int64_t)qi * kScoreHistBins, k, S, &bstar, &cgt, &ncand);
   if (bstar < 0 || ncand - cgt > kTieCap) return;  // topk_chunk_finish falls back
-  const int s0 = base + kPerThread * threadIdx.x;
-  const uint32_t word = scan32<kB16>(score_row<kB16>(scores, qi, ld), s0, n_t, bstar, gcount + qi,
-                                     gtidx + (int64_t)qi * kTieCap, gtkey + (int64_t)qi * kTieCap,
-                                     gh2 + (int64_t)qi * kSub);
-  if (s0 < n_t) gbits[(int64_t)qi * (ld / 32) + s0 / 32] = word;
+  // the chunk's bitmap words, up to the row's last word
+  const int n_words = min(kThreads, (n_t + 31) / 32 - base / 32);
+  scan_chunk<kB16>(score_row<kB16>(scores, qi, ld), base, n_t, bstar, gbits + (int64_t)qi * (ld / 32) + base / 32,
+                   n_words, gcount + qi, gtidx + (int64_t)qi * kTieCap, gtkey + (int64_t)qi * kTieCap,
+                   gh2 + (int64_t)qi * kSub);
 }
 
 // Histogram mode, longer rows, steps 3-4 per query.
@@ -461,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_chunk_finish(const void* __r
   }
   __syncthreads();
   uint32_t* rowbits = gbits + (int64_t)qi * (ld / 32);
-  resolve_ties<kB16>(nb, k - cgt, S, [&](int i) { atomicOr(rowbits + (i >> 5), 1u << (i & 31)); });
+  resolve_ties<kB16>(nb, k - cgt, n_t, S, [&](int i) { atomicOr(rowbits + (i >> 5), 1u << (i & 31)); });
   // output: each thread owns a contiguous run of bitmap words
   const int words = (n_t + 31) / 32;
   const int per = (words + kThreads - 1) / kThreads;
@@ -509,12 +587,28 @@ __global__ void __launch_bounds__(kThreads, 1) topk_staged(const void* __restric
     return;
   }
   StageSmem& S = *reinterpret_cast<StageSmem*>(smem_raw);
-  for (int s0 = kPerThread * threadIdx.x; s0 < n_t; s0 += kPerThread * kThreads) {
-    uint32_t keys[32];
-    ScoreKeys<kB16>::load32(row, s0, keys);
+  // coalesced 16-byte loads: 4 fp32 or 8 BF16 scores per thread per pass
+  constexpr int kPer = kB16 ? 8 : 4;
+  for (int s = kPer * threadIdx.x; s < n_t; s += kPer * kThreads) {
+    uint32_t kk[kPer];
+    if (kB16) {
+      const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(row) + s);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (s0 + e < n_t) S.ckey[s0 + e] = keys[e];
+      for (int j = 0; j < 4; ++j) {
+        kk[2 * j] = score_key16(w[j]);
+        kk[2 * j + 1] = score_key16(w[j] >> 16);
+      }
+    } else {
+      const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row) + s);
+      kk[0] = score_key(v.x);
+      kk[1] = score_key(v.y);
+      kk[2] = score_key(v.z);
+      kk[3] = score_key(v.w);
+    }
+#pragma unroll
+    for (int e = 0; e < kPer; ++e)
+      if (s + e < n_t) S.ckey[s + e] = kk[e];
   }
   __syncthreads();
   uint32_t thr;
