@@ -48,9 +48,10 @@
 // scale is outside that range, and logits that are not finite in fp32, are
 // dropped with CSA_DEV_ERR_RANGE.
 //
-// 8 warps (two per TMEM lane quadrant) gather, run the softmax and the
-// epilogue; thread 0 also issues the query TMA and the MMAs between block
-// barriers.  Every wait is bounded (CSA_DEV_ERR_TIMEOUT).
+// 16 warps (four per TMEM lane quadrant, 16 heads each) gather, convert
+// (warp w: row block w), run the softmax and the epilogue; thread 0 also
+// issues the query TMA and the MMAs between block barriers.  Every wait is
+// bounded (CSA_DEV_ERR_TIMEOUT).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -68,10 +69,12 @@ constexpr int kR = 64;
 constexpr int kNope = kD - kR;             // 448
 constexpr int kRowBytes = kNope + 2 * kR;  // 576
 constexpr int kChunks = kRowBytes / 16;    // 36 16-byte chunks per stored row
-constexpr int kThreads = 256;             // 8 warps: two per TMEM lane quadrant
-constexpr int kLoads = kRows * kChunks / kThreads;  // 18 loads per thread per tile
+constexpr int kThreads = 512;             // 16 warps: four per TMEM lane quadrant
+constexpr int kWarps = kThreads / 32;
+constexpr int kHPart = kHg / 4;           // heads per softmax / epilogue thread (16)
+constexpr int kLoads = kRows * kChunks / kThreads;  // 9 loads per thread per tile
 static_assert(kRows * kChunks % kThreads == 0, "gather must divide evenly");
-static_assert(kChunks == 36 && (kRows / 8) * (kChunks / 4) == 8 * kLoads, "conversion pairs cover the tile");
+static_assert(kChunks == 36 && kLoads == 9 && kRows / 8 == kWarps, "warp w converts row block w, chunk groups 0..8");
 constexpr float kLog2e = 1.4426950408889634f;
 // logits are kept in base-2 units (z * log2 e) so that probabilities are
 // exp2f of a difference; the running max is raised only when a tile exceeds
@@ -93,7 +96,7 @@ struct __align__(1024) AttnSmem {
   int live[kRows];            // row takes part (non-empty slot with a valid scale)
   uint32_t qamax[kHg];        // fp32 bits of each head's largest query magnitude
   float qg[kHg];              // 2^e_h: Q'_h = Q_h 2^-e_h
-  float red[8][64];
+  float red[kWarps][32];
   float mh[kHg], lh[kHg], alpha[kHg];
   float rope_c[kR / 2], rope_s[kR / 2];  // inverse-RoPE rotation of this query
   uint64_t bar_q, bar_g, bar_s, bar_o;
@@ -208,6 +211,26 @@ __device__ __forceinline__ float warp_transpose_reduce32(float (&v)[32]) {
   return v[0];
 }
 
+// max / sum over the 32 lanes of a warp for each of 16 values: afterwards
+// lane l holds the reduction of value index l % 16.
+template <bool kMax>
+__device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int s = 8; s >= 1; s >>= 1) {
+    const bool up = lane & s;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float keep = up ? v[i + s] : v[i];
+      const float send = up ? v[i] : v[i + s];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, s);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  const float o = __shfl_xor_sync(0xffffffffu, v[0], 16);
+  return kMax ? fmaxf(v[0], o) : v[0] + o;
+}
+
 // Row of candidate slot `slot` (< se) of query t: src 1 = cache row, 2 =
 // window ring row, 0 = empty; *off = element row index into that array.
 template <bool kDense>
@@ -247,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wt = threadIdx.x;                // 0..255
   const int quad = warp & 3;                 // TMEM lane quadrant of this warp
-  const int half = warp >> 2;                // head half: 32*half .. +31
+  const int part = warp >> 2;                // head part: 16*part .. +15
   const int j = quad * 32 + lane;            // tile row of this thread
   const int qi = blockIdx.x, split = blockIdx.y, hg = blockIdx.z;
   const int bs = qi / T, tq = qi % T;
@@ -356,24 +379,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     if (i == 0) {
       // each head's largest BF16 query magnitude (converted after the
       // barrier).  Word e of the query tile is head ((e >> 3) & 63): this
-      // thread's words belong to heads wt/8 (even steps) and wt/8 + 32 (odd)
+      // thread's words (e = wt + 512 n) all belong to head wt/8
       sm100::mbar_wait(&S.bar_q, 0, abort);
       const uint4* qv = reinterpret_cast<const uint4*>(&S.q[0][0]);
-      uint32_t ma = 0, mb = 0;
+      uint32_t ma = 0;
 #pragma unroll 4
-      for (int e = wt; e < 8 * kHg * 128 / 16; e += 2 * kThreads) {
-        ma = max(ma, bf16x8_amax_bits(qv[e]));
-        mb = max(mb, bf16x8_amax_bits(qv[e + kThreads]));
-      }
+      for (int e = wt; e < 8 * kHg * 128 / 16; e += kThreads) ma = max(ma, bf16x8_amax_bits(qv[e]));
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, o));
-        mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-      }
-      if ((lane & 7) == 0) {
-        atomicMax(&S.qamax[wt >> 3], ma << 16);
-        atomicMax(&S.qamax[(wt >> 3) + 32], mb << 16);
-      }
+      for (int o = 1; o < 8; o <<= 1) ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, o));
+      if ((lane & 7) == 0) atomicMax(&S.qamax[wt >> 3], ma << 16);
     }
     // Conversion work: (8-row block, group of four 16-byte chunks) pairs,
     // one pair per warp instruction, lane = 4 x row-in-block + chunk-in-group:
@@ -397,12 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       S.row_lc[wt] = log2f(cj);
       S.row_ic[wt] = 1.f / cj;
     }
-    // Pair k of this warp: chunk group k % 9 (compile-time: groups 0-6 are
-    // E4M3 codes, 7-8 RoPE dims) of 8-row block warp + 8 (k / 9).
+    // Pair k of this warp: chunk group k (compile-time: groups 0-6 are E4M3
+    // codes, 7-8 RoPE dims) of 8-row block `warp`.
     uint4 raw[kLoads];
 #pragma unroll
     for (int k = 0; k < kLoads; ++k) {
-      const int r = 8 * (warp + 8 * (k / 9)) + (lane >> 2), c = 4 * (k % 9) + (lane & 3);
+      const int r = 8 * warp + (lane >> 2), c = 4 * k + (lane & 3);
       raw[k] = *reinterpret_cast<const uint4*>(stg + r * kRowBytes + c * 16);
     }
     __syncthreads();  // staging area read by all; row factors, live flags, query amax visible
@@ -415,21 +429,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       };
       if (wt < kHg) S.qg[wt] = __uint_as_float((uint32_t)(127 + head_exp(wt)) << 23);
       const float qia = __uint_as_float((uint32_t)(127 - head_exp(wt >> 3)) << 23);
-      const float qib = __uint_as_float((uint32_t)(127 - head_exp((wt >> 3) + 32)) << 23);
       uint4* qv = reinterpret_cast<uint4*>(&S.q[0][0]);
 #pragma unroll 4
-      for (int e = wt; e < 8 * kHg * 128 / 16; e += 2 * kThreads) {
-        qv[e] = bf16x8_scale_to_f16(qv[e], qia);
-        qv[e + kThreads] = bf16x8_scale_to_f16(qv[e + kThreads], qib);
-      }
+      for (int e = wt; e < 8 * kHg * 128 / 16; e += kThreads) qv[e] = bf16x8_scale_to_f16(qv[e], qia);
     }
     // -- convert + store V' (empty and dropped rows as zeros: the staging
     //    area holds stale bytes there)
 #pragma unroll
     for (int k = 0; k < kLoads; ++k) {
-      const int r = 8 * (warp + 8 * (k / 9)) + (lane >> 2), c = 4 * (k % 9) + (lane & 3);
+      const int r = 8 * warp + (lane >> 2), c = 4 * k + (lane & 3);
       const bool live = S.live[r] != 0;
-      if (k % 9 < kNope / 64) {
+      if (k < kNope / 64) {
         // dims 16c .. 16c+15 -> K-chunk (16c)/64, 16-byte slots 2(c%4), 2(c%4)+1;
         // codes times 2^k (exact down to 2^-24)
         uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
@@ -490,42 +500,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     sm100::mbar_wait(&S.bar_s, i & 1, abort);
     sm100::tc_fence_after();
     // -- this thread's row: c_j = s_j 2^-k_j, and u = z + log2 c_j (base-2
-    //    logit plus the row's log-scale) for its 32 heads
+    //    logit plus the row's log-scale) for its 16 heads
     const float inv_c = S.row_ic[j];  // 1 / c_j
-    float z[32];
+    float z[kHPart];
     {
-      uint32_t a[16], b[16];
-      const uint32_t ta = s_col + ((uint32_t)(quad * 32) << 16) + 32 * half;
-      sm100::tmem_ld_x16(ta, a);
-      sm100::tmem_ld_x16(ta + 16, b);
+      uint32_t a[16];
+      sm100::tmem_ld_x16(s_col + ((uint32_t)(quad * 32) << 16) + kHPart * part, a);
       sm100::tmem_ld_wait();
       const bool valid = S.live[j] != 0;
       const float f = S.row_f[j];
       const float lc = S.row_lc[j];
       bool bad = false;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float za = f * S.qg[32 * half + c] * __uint_as_float(a[c]);
-        const float zb = f * S.qg[32 * half + 16 + c] * __uint_as_float(b[c]);
-        const bool ba = !(fabsf(za) < INFINITY), bb = !(fabsf(zb) < INFINITY);
-        bad |= valid && (ba || bb);
+      for (int c = 0; c < kHPart; ++c) {
+        const float za = f * S.qg[kHPart * part + c] * __uint_as_float(a[c]);
+        const bool ba = !(fabsf(za) < INFINITY);
+        bad |= valid && ba;
         z[c] = (valid && !ba) ? za + lc : -INFINITY;
-        z[16 + c] = (valid && !bb) ? zb + lc : -INFINITY;
       }
       if (bad) raise_err(err, CSA_DEV_ERR_RANGE);  // a logit beyond fp32: dropped
     }
     // per-head tile maxima
     {
-      float v[32];
+      float v[kHPart];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] = z[c];
-      S.red[warp][lane] = warp_transpose_reduce32<true>(v);  // head 32*half + lane, this warp's rows
+      for (int c = 0; c < kHPart; ++c) v[c] = z[c];
+      S.red[warp][lane] = warp_transpose_reduce16<true>(v);  // head 16*part + lane%16, this warp's rows
     }
     __syncthreads();
     if (wt < kHg) {
-      const int h = wt, hh = h >> 5, hl = h & 31;
+      const int h = wt, hp = h / kHPart, hl = h % kHPart;
       float tmax = -INFINITY;
-      for (int q4 = 0; q4 < 4; ++q4) tmax = fmaxf(tmax, S.red[hh * 4 + q4][hl]);
+      for (int q4 = 0; q4 < 4; ++q4) tmax = fmaxf(tmax, S.red[4 * hp + q4][hl]);
       const float mo = S.mh[h];
       float al = 1.f;
       int resc = 0;
@@ -546,47 +552,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     if (i > 0 && S.rescale) {
 #pragma unroll 1
       for (int blk = 0; blk < 4; ++blk) {
+        uint32_t r16[16];
+        const uint32_t ta = o_col + 64 * blk + ((uint32_t)(quad * 32) << 16) + kHPart * part;
+        sm100::tmem_ld_x16(ta, r16);
+        sm100::tmem_ld_wait();
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          uint32_t r16[16];
-          const uint32_t ta = o_col + 64 * blk + ((uint32_t)(quad * 32) << 16) + 32 * half + 16 * g;
-          sm100::tmem_ld_x16(ta, r16);
-          sm100::tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            r16[c] = __float_as_uint(__uint_as_float(r16[c]) * S.alpha[32 * half + 16 * g + c]);
-          sm100::tmem_st_x16(ta, r16);
-        }
+        for (int c = 0; c < 16; ++c) r16[c] = __float_as_uint(__uint_as_float(r16[c]) * S.alpha[kHPart * part + c]);
+        sm100::tmem_st_x16(ta, r16);
       }
       sm100::tmem_st_wait();
     }
-    // P' = exp2(u - m_h) (FP16 stores: row j, heads 32*half .. +31 = four
+    // P' = exp2(u - m_h) (FP16 stores: row j, heads 16*part .. +15 = two
     // 16-byte words) and the per-head sums of exp2(z - m_h) = P' / c_j
     {
-      float v[32];
+      float v[kHPart];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float mh = S.mh[32 * half + c];
+      for (int c = 0; c < kHPart; ++c) {
+        const float mh = S.mh[kHPart * part + c];
         v[c] = (mh == -INFINITY || z[c] == -INFINITY) ? 0.f : exp2f(z[c] - mh);
       }
 #pragma unroll
-      for (int w4 = 0; w4 < 4; ++w4) {
-        const int b = 8 * w4;
+      for (int w2 = 0; w2 < 2; ++w2) {
+        const int b = 8 * w2;
         const uint4 pk = make_uint4(pack_half2(v[b], v[b + 1]), pack_half2(v[b + 2], v[b + 3]),
                                     pack_half2(v[b + 4], v[b + 5]), pack_half2(v[b + 6], v[b + 7]));
-        *reinterpret_cast<uint4*>(S.p + sw128(j, 4 * half + w4)) = pk;
+        *reinterpret_cast<uint4*>(S.p + sw128(j, 2 * part + w2)) = pk;
       }
 #pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] *= inv_c;
-      S.red[warp][lane] = warp_transpose_reduce32<false>(v);
+      for (int c = 0; c < kHPart; ++c) v[c] *= inv_c;
+      S.red[warp][lane] = warp_transpose_reduce16<false>(v);
     }
     sm100::tc_fence_before();
     sm100::fence_proxy_async_smem();
     __syncthreads();
     if (wt < kHg) {
-      const int h = wt, hh = h >> 5, hl = h & 31;
+      const int h = wt, hp = h / kHPart, hl = h % kHPart;
       float ts = 0.f;
-      for (int q4 = 0; q4 < 4; ++q4) ts += S.red[hh * 4 + q4][hl];
+      for (int q4 = 0; q4 < 4; ++q4) ts += S.red[4 * hp + q4][hl];
       S.lh[h] += ts;
     }
     // -- O^T[blk] += V'^T[blk] P' over K = 128 rows (8 steps of 16)
@@ -634,24 +636,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   __syncthreads();
   const bool ok = !S.abort;
   if (ok && n_tiles > 0) {
-    float f[32];
+    float f[kHPart];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) f[c] = S.alpha[32 * half + c];
+    for (int c = 0; c < kHPart; ++c) f[c] = S.alpha[kHPart * part + c];
     // [64 heads][512 dims]: BF16 output, or the fp32 partial (128 KB, all of V')
     uint16_t* stage = reinterpret_cast<uint16_t*>(&S.v[0][0]);
     float* stage32 = reinterpret_cast<float*>(&S.v[0][0]);
 #pragma unroll 1
     for (int b2 = 0; b2 < 4; b2 += 2) {
-      // four TMEM loads in flight: blocks b2, b2+1, this warp's 32 heads
-      uint32_t rr[4][16];
+      // two TMEM loads in flight: blocks b2, b2+1, this warp's 16 heads
+      uint32_t rr[2][16];
 #pragma unroll
-      for (int x = 0; x < 4; ++x)
-        sm100::tmem_ld_x16(o_col + 64 * (b2 + (x >> 1)) + ((uint32_t)(quad * 32) << 16) + 32 * half + 16 * (x & 1),
-                           rr[x]);
+      for (int x = 0; x < 2; ++x)
+        sm100::tmem_ld_x16(o_col + 64 * (b2 + x) + ((uint32_t)(quad * 32) << 16) + kHPart * part, rr[x]);
       sm100::tmem_ld_wait();
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int blk = b2 + (x >> 1), g = x & 1;
+      for (int x = 0; x < 2; ++x) {
+        const int blk = b2 + x;
         const int c_dim = 128 * blk + quad * 32 + lane;
         float cs = 1.f, sn = 0.f;
         if (single && c_dim >= kNope) {
@@ -660,10 +661,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
         }
         const bool odd = lane & 1;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int hl = 16 * g + c;
-          const int h = 32 * half + hl;
-          float y = __uint_as_float(rr[x][c]) * f[hl];
+        for (int c = 0; c < kHPart; ++c) {
+          const int h = kHPart * part + c;
+          float y = __uint_as_float(rr[x][c]) * f[c];
           if (single) {
             const float pv = __shfl_xor_sync(0xffffffffu, y, 1);
             if (c_dim >= kNope) y = odd ? (pv * sn + y * cs) : (y * cs - pv * sn);
