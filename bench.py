@@ -468,6 +468,9 @@ def main():
                     help="device copies rotated in the timed loop (0: enough to exceed 3x L2)")
     ap.add_argument("--score-fmt", default="f32", choices=["f32", "bf16"],
                     help="index-score precision the selector ranks (bf16: the BF16-score variant)")
+    ap.add_argument("--prefill-len", type=int, default=0,
+                    help="c4 only: a shorter prefill (L = T = this many tokens per sequence) for profiling "
+                         "small cases; 0 keeps the workload's 32768")
     ap.add_argument("--extra-configs", default="c2,c3,c4",
                     help="with --config c1 on one GPU: the other workloads measured into the same line")
     args = ap.parse_args()
@@ -516,13 +519,77 @@ def main():
         dist.destroy_process_group()
 
 
+def bf16_score_entry(w, dw32, stream, reps=20):
+    """The BF16-score variant of the index call on the same inputs (kwkr.cn
+    notes 4.4: index scores quantised from FP32 to BF16 before the top-k
+    selector): its mean event time beside the fp32 call's, and how much of
+    the fp32-score top-k set the BF16-score selection keeps (mean over the
+    batch's queries).  Both sets are exact (tests compare each with the
+    oracle's selection), so this is the recall of the method, not of the
+    kernels."""
+    import torch
+    from long_context_sparse_gated_b200.runner import DeviceWorkload
+    dw16 = DeviceWorkload(synth.with_score_fmt(w, "bf16"))
+
+    def timed(dw):
+        for _ in range(3):
+            dw.index_topk()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            dw.index_topk()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return float(np.median(ts)) * 1e3
+
+    us32, us16 = timed(dw32), timed(dw16)
+    i32 = dw32.idx.cpu().numpy().reshape(-1, dw32.idx.shape[-1])
+    i16 = dw16.idx.cpu().numpy().reshape(-1, dw16.idx.shape[-1])
+    rec = []
+    for a, b in zip(i32, i16):
+        sa = set(a[a >= 0].tolist())
+        rec.append(len(sa & set(b[b >= 0].tolist())) / max(len(sa), 1))
+    del dw16
+    return {"index_call_us_fp32": us32, "index_call_us_bf16": us16,
+            "recall_of_fp32_topk": float(np.mean(rec)), "recall_min": float(np.min(rec)),
+            "how": "host-launched index calls on one device copy, median of 20 event-timed calls each; "
+                   "recall = |BF16-score top-k & fp32-score top-k| / min(k, n_t), mean over the queries"}
+
+
+def host_call_us(dw, reps=100):
+    """Host time per public call through the Python binding: the mean wall
+    time of `reps` back-to-back calls, with the device work queued behind
+    and not waited for (argument checks, cached driver work, launches)."""
+    import torch
+    calls = {"csa_compress" if dw.p.m < 64 else "hca_compress": dw.compress}
+    if dw.p.k > 0:
+        calls.update({"csa_index_topk": dw.index_topk, "csa_sparse_attn": dw.sparse_attn})
+    else:
+        calls["hca_dense_attn"] = dw.dense_attn
+    out = {}
+    for name, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        t = time.perf_counter()
+        for _ in range(reps):
+            fn()
+        out[name] = (time.perf_counter() - t) / reps * 1e6
+        torch.cuda.synchronize()
+    out["how"] = f"mean wall time of {reps} back-to-back host calls, device work not awaited"
+    return out
+
+
 def run_config(config, args, world, rank, local):
     """Measure one workload; rank 0 returns its JSON entry, others None."""
     import torch
     import torch.distributed as dist
     from long_context_sparse_gated_b200.runner import STEP_INPUTS, DeviceWorkload
 
-    w = synth.with_score_fmt(synth.config(config, seed=rank_seed(config, rank)), args.score_fmt)
+    over = {"L": args.prefill_len} if config == "c4" and args.prefill_len > 0 else {}
+    w = synth.with_score_fmt(synth.config(config, seed=rank_seed(config, rank), **over), args.score_fmt)
     step_bytes, idx_bytes = algorithmic_bytes(w)
     n_copies = max(1, int(np.ceil(3 * L2_BYTES / step_bytes)))
     if config == "c4":
@@ -727,7 +794,8 @@ def run_config(config, args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8/bf16 storage, mxfp4 indexer, fp32 accumulate" if p.kv_fmt == "fp8" else "f32",
         "data": "synthetic",
-        "config": {"workload": CONFIG_NAMES[config], "name": config, "batch": p.B, "index_scores": args.score_fmt,
+        "config": {"workload": CONFIG_NAMES[config] + (f", reduced to L = T = {args.prefill_len}" if over else ""),
+                   "name": config, "batch": p.B, "index_scores": args.score_fmt,
                    "context": int(w["L"].max()), "queries_per_step": queries,
                    "l2": f"inputs larger than L2: {n_copies} device copies rotated, {n_copies * step_bytes / 2**20:.0f} MiB per cycle"},
         "gpu_launches": args.steps * (kernels_per_step if kernels_per_step is not None else launches_per_step(w)),
@@ -740,6 +808,10 @@ def run_config(config, args, world, rank, local):
         "clocks": clocks,
         "device_err_bits": err,
     }
+    if world == 1:
+        line["host_us_per_call"] = host_call_us(dws[0], reps=100 if queries <= 4096 else 10)
+    if p.k > 0 and w["T"] <= 4 and args.score_fmt == "f32" and world == 1:
+        line["bf16_scores"] = bf16_score_entry(w, dws[0], stream)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline_entry(w, config)
     del dws

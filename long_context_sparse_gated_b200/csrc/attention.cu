@@ -296,7 +296,7 @@ static cudaError_t launch_attn_t(const csa_params& p, const void* q, const csa_k
   const int nhg = (p.n_heads + kHeadGroup - 1) / kHeadGroup;
   const size_t smem = attn_smem_bytes(p.d);
   auto kfn = attn_split_simt<kKvF32, kActF32, kDense>;
-  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(kfn), smem);
   if (e != cudaSuccess) return e;
   Rows rc{reinterpret_cast<const uint8_t*>(cache.rows), cache.scale, cache.cap};
   Rows rw{reinterpret_cast<const uint8_t*>(win.rows), win.scale, win.cap};

@@ -32,9 +32,20 @@
 //              which is added to the global per-query histogram (the top-k
 //              selector's starting point) when the warpgroup moves to
 //              another query and at the end
-// Each CTA walks a contiguous range of (query, 256-entry block) stages, so
-// the key stream it reads is sequential.  Stages past a query's n_t are
-// skipped.
+// Two ways of walking the work, chosen by the host from the call's shape:
+//   decode (T <= 4): a stage is 256 entries of one query (two 128-entry
+//       MMA tiles, N = 64 heads); each CTA walks a contiguous range of
+//       (query, stage) pairs, so the key stream it reads is sequential and
+//       a long row is spread over many CTAs.  Stages past n_t are skipped.
+//   prefill (T > 4): a stage is 128 entries of a pair of consecutive
+//       queries of one sequence (one MMA tile with N = 128: both queries'
+//       64 heads), so every key tile read from L2 serves two queries and
+//       each MMA is twice as wide.  CTA b takes query pairs b, b + grid,
+//       ... with all their visible stages, which balances the causal
+//       (growing) rows over the CTAs.  Epilogue warpgroup g takes query g
+//       of the pair.
+// In both modes an accumulator is 128 TMEM columns and each epilogue
+// warpgroup reads 64 of them per stage.
 //
 // Numerics: with MXFP4 inputs whose per-32 scales are >= 2^-2 and dyadic
 // head weights, every partial sum is exactly representable in fp32 (the
@@ -59,8 +70,6 @@ constexpr int kKeyBytes = kTileM * kRowBytes;   // 8192 per tile
 constexpr int kQBytes = kHeads * kRowBytes;     // 4096
 constexpr int kSfkBytes = kTileM * 4;           // 512 per tile (4 UE8M0 per row)
 constexpr int kSfqBytes = kHeads * 4;           // 256
-constexpr uint32_t kStageTx = kTiles * (kKeyBytes + kSfkBytes);
-constexpr uint32_t kQueryTx = kQBytes + kSfqBytes;
 
 // A tile's 128 keys are loaded through a 3-D view of the key array, so that
 // MMA row 32q + i holds key 4i + q (q < 4, i < 32).  With that order the
@@ -72,10 +81,12 @@ struct __align__(1024) Stage {
   uint32_t sfk[kTiles][kTileM];     // the stage's 256 scale words, in entry order
 };
 
+constexpr int kPair = 2;       // queries per stage in prefill mode
+
 struct __align__(1024) QuerySlot {
-  uint8_t q[kQBytes];
-  uint32_t sfq_raw[kHeads];
-  uint32_t sfq[kTileM];     // permuted for tcgen05.cp; rows 64..127 zero
+  uint8_t q[kPair * kQBytes];         // one query (decode) or a pair (prefill)
+  uint32_t sfq_raw[kPair * kHeads];
+  uint32_t sfq[kTileM];     // permuted for tcgen05.cp (decode: rows 64..127 zero)
 };
 
 constexpr int kAcc = 3;         // TMEM accumulator pairs (one tile each per epilogue warpgroup)
@@ -96,8 +107,9 @@ struct Smem {
   int abort;
 };
 
-// TMEM columns: accumulator pair a, tile g at 128 a + 64 g (0..383); key
-// scales 384 + 8 a + 4 g; query scales 408 + 4 slot.
+// TMEM columns: accumulator a at 128 a (0..383): decode tile g at
+// 128 a + 64 g, prefill query g at 128 a + 64 g; key scales 384 + 8 a + 4 g;
+// query scales 408 + 4 slot.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfaCol = kAcc * kTiles * kHeads;
 constexpr uint32_t kSfbCol = kSfaCol + 4 * kTiles * kAcc;
@@ -109,52 +121,118 @@ __device__ __forceinline__ int visible(const int32_t* q_pos0, int T, int m, int 
   return (int)(n < n_max ? n : n_max);
 }
 
-// visible() of the current query, re-read only when the query changes: the
-// single producer thread must not pay a global-load latency per tile.
-struct VisibleCache {
-  int qi = -1, n = 0;
-  __device__ __forceinline__ int get(const int32_t* q_pos0, int T, int m, int q, int n_max) {
-    if (q != qi) {
-      qi = q;
-      n = visible(q_pos0, T, m, q, n_max);
-    }
-    return n;
-  }
-};
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory per CTA");
 
 constexpr int kThreadsTc = 64 + 128 * kEpiGroups;  // producer, MMA, 2 epilogue warpgroups
 
-// Walks the CTA's tile range as (query, block) pairs.  One 64-bit division
-// at the start; afterwards a step is an increment, so the single-thread
-// producer and MMA loops do not pay a division latency per tile.
-struct TileCursor {
+// Shape of one walking mode (see the header).
+template <bool kPrefill>
+struct Mode {
+  static constexpr int kQn = kPrefill ? kPair : 1;          // queries per stage
+  static constexpr int kT = kPrefill ? 1 : kTiles;          // MMA tiles per stage
+  static constexpr int kKeys = kT * kTileM;                 // entries per stage
+  static constexpr int kN = kQn * kHeads;                   // MMA N
+  static constexpr uint32_t kStageTx = kT * (kKeyBytes + kSfkBytes);
+  static constexpr uint32_t kQueryTx = kQn * (kQBytes + kSfqBytes);
+};
+
+// The stages one CTA walks, in order.  After next() returns true: q0 is
+// the stage's first query, j its stage index within the row, nvis the
+// visible entries of the stage's last query, and fresh is set when the
+// query (pair) differs from the previous stage's.
+template <bool kPrefill>
+struct Walker;
+
+// decode: a contiguous range of (query, 256-entry stage) pairs.  One 64-bit
+// division at the start; afterwards a step is an increment, so the
+// single-thread producer and MMA loops do not pay a division latency per
+// stage.  visible() is re-read only when the query changes.
+template <>
+struct Walker<false> {
   int64_t t, end;
-  int qi, j, tpq;
-  __device__ __forceinline__ TileCursor(int64_t begin, int64_t e, int tiles_per_query)
-      : t(begin), end(e), tpq(tiles_per_query) {
-    qi = (int)(begin / tiles_per_query);
-    j = (int)(begin - (int64_t)qi * tiles_per_query);
+  int qi, jj, tpq;
+  int q0 = -1, j = 0, nvis = 0;
+  bool fresh = false;
+  __device__ __forceinline__ Walker(int n_queries, int n_max) {
+    tpq = (n_max + Mode<false>::kKeys - 1) / Mode<false>::kKeys;
+    const int64_t n_units = (int64_t)n_queries * tpq;
+    t = n_units * blockIdx.x / gridDim.x;
+    end = n_units * (blockIdx.x + 1) / gridDim.x;
+    qi = (int)(t / tpq);
+    jj = (int)(t - (int64_t)qi * tpq);
   }
-  __device__ __forceinline__ bool more() const { return t < end; }
-  __device__ __forceinline__ void next() {
-    ++t;
-    if (++j == tpq) { j = 0; ++qi; }
+  __device__ __forceinline__ bool next(const int32_t* q_pos0, int T, int m, int n_max) {
+    while (t < end) {
+      const int q = qi, js = jj;
+      ++t;
+      if (++jj == tpq) { jj = 0; ++qi; }
+      const bool nq = q != q0;
+      if (nq) nvis = visible(q_pos0, T, m, q, n_max);
+      if (js * Mode<false>::kKeys >= nvis) {
+        if (nq) { q0 = q; fresh_pending = true; }
+        continue;
+      }
+      fresh = nq || fresh_pending;
+      fresh_pending = false;
+      q0 = q;
+      j = js;
+      return true;
+    }
+    return false;
+  }
+  bool fresh_pending = false;
+};
+
+// prefill: query pairs b, b + grid, ... of the batch (pairs never cross a
+// sequence), each with all of its visible 128-entry stages.
+template <>
+struct Walker<true> {
+  int g, n_groups, gps;
+  int q0 = 0, qn = 0, j = 0, nst = 0, nvis = 0;
+  bool fresh = false;
+  __device__ __forceinline__ Walker(int n_queries, int T) {
+    gps = (T + kPair - 1) / kPair;
+    n_groups = (n_queries / T) * gps;
+    g = (int)blockIdx.x - (int)gridDim.x;
+  }
+  __device__ __forceinline__ bool next(const int32_t* q_pos0, int T, int m, int n_max) {
+    if (++j < nst) {
+      fresh = false;
+      return true;
+    }
+    while (true) {
+      g += gridDim.x;
+      if (g >= n_groups) return false;
+      const int bs = g / gps, tq = kPair * (g - bs * gps);
+      q0 = bs * T + tq;
+      qn = T - tq < kPair ? T - tq : kPair;
+      nvis = visible(q_pos0, T, m, q0 + qn - 1, n_max);
+      nst = (nvis + Mode<true>::kKeys - 1) / Mode<true>::kKeys;
+      if (nst > 0) break;
+    }
+    j = 0;
+    fresh = true;
+    return true;
   }
 };
 
+template <bool kPrefill>
+__device__ __forceinline__ Walker<kPrefill> make_walker(int n_queries, int T, int n_max) {
+  if constexpr (kPrefill) return Walker<true>(n_queries, T);
+  else return Walker<false>(n_queries, n_max);
+}
+
+template <bool kPrefill>
 __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     const __grid_constant__ CUtensorMap tm_key, const __grid_constant__ CUtensorMap tm_q,
     const __grid_constant__ CUtensorMap tm_sfk, const __grid_constant__ CUtensorMap tm_sfq,
     const float* __restrict__ w, const int32_t* __restrict__ q_pos0, int T, int m, int64_t k_cap,
     int n_queries, int n_max, void* __restrict__ scores, int ld, int b16, uint32_t* __restrict__ hist,
     int32_t* __restrict__ err) {
+  using M = Mode<kPrefill>;
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tpq = (n_max + kStageKeys - 1) / kStageKeys;  // stages per query
-  const int64_t n_tiles = (int64_t)n_queries * tpq;
-  const int64_t t_begin = n_tiles * blockIdx.x / gridDim.x;
-  const int64_t t_end = n_tiles * (blockIdx.x + 1) / gridDim.x;
   volatile int* abort = &S.abort;
 
   if (threadIdx.x == 0) {
@@ -191,30 +269,27 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       sm100::prefetch_tmap(&tm_sfk);
       sm100::prefetch_tmap(&tm_sfq);
       uint32_t it = 0, nq = 0;
-      int cur_q = -1;
-      VisibleCache vc;
       int bs = 0;
-      for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
-        const int qi = c.qi, j = c.j;
-        if (j * kStageKeys >= vc.get(q_pos0, T, m, qi, n_max)) continue;
-        if (qi != cur_q) {  // the query's 64 heads, once per query
-          bs = qi / T;
+      auto wk = make_walker<kPrefill>(n_queries, T, n_max);
+      while (wk.next(q_pos0, T, m, n_max)) {
+        if (wk.fresh) {  // the stage's query (pair): 64 heads each, once per query
+          bs = wk.q0 / T;
           const int sl = nq & 1;
           if (!sm100::mbar_wait(&S.qempty[sl], ((nq >> 1) & 1) ^ 1, abort)) break;
-          sm100::mbar_arrive_expect_tx(&S.qfull[sl], kQueryTx);
-          sm100::tma_load_2d(S.qs[sl].q, &tm_q, &S.qfull[sl], 0, qi * kHeads);
-          sm100::tma_load_1d(S.qs[sl].sfq_raw, &tm_sfq, &S.qfull[sl], qi * kHeads);
-          cur_q = qi;
+          sm100::mbar_arrive_expect_tx(&S.qfull[sl], M::kQueryTx);
+          sm100::tma_load_2d(S.qs[sl].q, &tm_q, &S.qfull[sl], 0, wk.q0 * kHeads);
+          sm100::tma_load_1d(S.qs[sl].sfq_raw, &tm_sfq, &S.qfull[sl], wk.q0 * kHeads);
           ++nq;
         }
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!sm100::mbar_wait(&S.empty[s], ph ^ 1, abort)) break;
         Stage& st = S.st[s];
-        sm100::mbar_arrive_expect_tx(&S.full[s], kStageTx);
-        const int64_t row = (int64_t)bs * k_cap + (int64_t)j * kStageKeys;
-        sm100::tma_load_3d(st.key[0], &tm_key, &S.full[s], 0, (int32_t)(row / 4), 0);
-        sm100::tma_load_3d(st.key[1], &tm_key, &S.full[s], 0, (int32_t)(row / 4) + kTileM / 4, 0);
+        sm100::mbar_arrive_expect_tx(&S.full[s], M::kStageTx);
+        const int64_t row = (int64_t)bs * k_cap + (int64_t)wk.j * M::kKeys;
+#pragma unroll
+        for (int g = 0; g < M::kT; ++g)
+          sm100::tma_load_3d(st.key[g], &tm_key, &S.full[s], 0, (int32_t)(row / 4) + g * (kTileM / 4), 0);
         sm100::tma_load_1d(st.sfk, &tm_sfk, &S.full[s], (int32_t)row);
         ++it;
       }
@@ -223,25 +298,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     // ---------------- MMA issuer (one lane) ----------------
     if (lane == 0) {
       uint32_t it = 0, nq = 0;
-      int cur_q = -1, sl = 0;
-      VisibleCache vc;
-      for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
-        const int qi = c.qi, j = c.j;
-        if (j * kStageKeys >= vc.get(q_pos0, T, m, qi, n_max)) continue;
-        if (qi != cur_q) {
+      int sl = 0;
+      auto wk = make_walker<kPrefill>(n_queries, T, n_max);
+      while (wk.next(q_pos0, T, m, n_max)) {
+        if (wk.fresh) {
           // the previous query's slot is free once its MMAs complete
-          if (cur_q >= 0) sm100::tc_commit(&S.qempty[sl]);
+          if (nq > 0) sm100::tc_commit(&S.qempty[sl]);
           sl = nq & 1;
           if (!sm100::mbar_wait(&S.qfull[sl], (nq >> 1) & 1, abort)) break;
-          // query scales: head h's word goes to line h%32, slot h/32
+          // query scales: MMA column n's word goes to line n % 32, word n / 32
           QuerySlot& qs = S.qs[sl];
 #pragma unroll 4
           for (int l = 0; l < 32; ++l)
-            reinterpret_cast<uint4*>(qs.sfq)[l] = make_uint4(qs.sfq_raw[l], qs.sfq_raw[l + 32], 0u, 0u);
+            reinterpret_cast<uint4*>(qs.sfq)[l] =
+                kPrefill ? make_uint4(qs.sfq_raw[l], qs.sfq_raw[l + 32], qs.sfq_raw[l + 64], qs.sfq_raw[l + 96])
+                         : make_uint4(qs.sfq_raw[l], qs.sfq_raw[l + 32], 0u, 0u);
           sm100::fence_proxy_async_smem();
           sm100::tc_fence_after();
           sm100::tc_cp_32x128b_warpx4(tmem + kSfbCol + 4 * sl, sm100::smem_desc(sm100::smem_u32(qs.sfq), 0, 128, 0));
-          cur_q = qi;
           ++nq;
         }
         const int s = it % kStages;
@@ -254,8 +328,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         const uint32_t sfb_col = tmem + kSfbCol + 4 * sl;
         const uint32_t qa = sm100::smem_u32(S.qs[sl].q);
 #pragma unroll
-        for (int g = 0; g < kTiles; ++g) {
-          const uint32_t d_col = tmem + (acc * kTiles + g) * kHeads;
+        for (int g = 0; g < M::kT; ++g) {
+          const uint32_t d_col = tmem + acc * kTiles * kHeads + g * kHeads;
           const uint32_t sfa_col = tmem + kSfaCol + 4 * (acc * kTiles + g);
           sm100::tc_cp_32x128b_warpx4(sfa_col, sm100::smem_desc(sm100::smem_u32(st.sfk[g]), 0, 128, 0));
           const uint32_t ka = sm100::smem_u32(st.key[g]);
@@ -264,12 +338,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
             // K elements [64kk, 64kk+64) = bytes [32kk, 32kk+32) of every row
             const uint64_t adesc = sm100::smem_desc(ka + 32 * kk, 16, 512, 4);
             const uint64_t bdesc = sm100::smem_desc(qa + 32 * kk, 16, 512, 4);
-            sm100::mma_mxf4(d_col, adesc, bdesc, sm100::idesc_mxf4(kTileM, kHeads, 2 * kk, 2 * kk), sfa_col,
+            sm100::mma_mxf4(d_col, adesc, bdesc, sm100::idesc_mxf4(kTileM, M::kN, 2 * kk, 2 * kk), sfa_col,
                             sfb_col, kk);
           }
         }
-        // completion: the accumulator pair is ready for the epilogue, and
-        // the stage's shared memory goes back to the producer
+        // completion: the accumulator is ready for the epilogue, and the
+        // stage's shared memory goes back to the producer
         sm100::tc_commit(&S.tfull[acc]);
         sm100::tc_commit(&S.empty[s]);
         ++it;
@@ -277,7 +351,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
     }
   } else {
     // ---------------- epilogue (warps 2..9: two warpgroups) ----------------
-    const int eg = (warp - 2) >> 2;  // warpgroup: tile eg of every stage
+    const int eg = (warp - 2) >> 2;  // warpgroup: tile (decode) or query (prefill) eg of every stage
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     // TMEM lane 32*quad + lane holds key 4*lane + quad of the tile
     const int key_in_tile = 4 * lane + quad;
@@ -300,30 +374,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       sm100::named_bar_sync(1 + eg, 128);
     }
     uint32_t it = 0;
-    int wq = -1;
+    int wq = -1, n_t = 0;
     float wv[kHeads];
-    VisibleCache vc;
-    for (TileCursor c(t_begin, t_end, tpq); c.more(); c.next()) {
-      const int qi = c.qi, j = c.j;
-      const int n_t = vc.get(q_pos0, T, m, qi, n_max);
-      if (j * kStageKeys >= n_t) continue;
+    auto wk = make_walker<kPrefill>(n_queries, T, n_max);
+    while (wk.next(q_pos0, T, m, n_max)) {
       const uint32_t my = it++;
       const int acc = my % kAcc;
       const uint32_t aph = (my / kAcc) & 1;
-      if (qi != wq) {  // head weights of this tile's query, kept in registers
+      if (wk.fresh) {  // this warpgroup's query changed: flush, load its head weights
         if (hist && wq >= 0) flush(wq);
-        const float4* wp = reinterpret_cast<const float4*>(w + (int64_t)qi * kHeads);
-#pragma unroll
-        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
-          const float4 v = __ldg(wp + h4);
-          wv[4 * h4] = v.x; wv[4 * h4 + 1] = v.y; wv[4 * h4 + 2] = v.z; wv[4 * h4 + 3] = v.w;
+        int q = wk.q0;
+        n_t = wk.nvis;
+        if constexpr (kPrefill) {
+          q = eg < wk.qn ? wk.q0 + eg : -1;
+          n_t = q >= 0 ? visible(q_pos0, T, m, q, n_max) : 0;
         }
-        wq = qi;
+        if (q >= 0) {
+          const float4* wp = reinterpret_cast<const float4*>(w + (int64_t)q * kHeads);
+#pragma unroll
+          for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+            const float4 v = __ldg(wp + h4);
+            wv[4 * h4] = v.x; wv[4 * h4 + 1] = v.y; wv[4 * h4 + 2] = v.z; wv[4 * h4 + 3] = v.w;
+          }
+        }
+        wq = q;
       }
       int ok = 1;
       if (lane == 0) ok = sm100::mbar_wait(&S.tfull[acc], aph, abort);
       // no break on a failed wait: every warp of the warpgroup keeps walking
-      // the same tiles so that the histogram flushes' named barriers match;
+      // the same stages so that the histogram flushes' named barriers match;
       // after an abort every wait returns at once and no work is done
       if (!__shfl_sync(0xffffffffu, ok, 0)) continue;
       sm100::tc_fence_after();
@@ -343,16 +422,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
 #pragma unroll
       for (int h = 0; h < kHeads; ++h) p4[h & 3] = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), p4[h & 3]);
       const float sc = (p4[0] + p4[1]) + (p4[2] + p4[3]);
-      const int s_idx = j * kStageKeys + eg * kTileM + key_in_tile;
+      const int s_idx = wk.j * M::kKeys + (kPrefill ? 0 : eg * kTileM) + key_in_tile;
       if (s_idx < n_t) {
         // fp32 score, or rounded to BF16 (nearest even) for the BF16
         // selector; the histogram bins the key the selector will rank
         if (b16) {
           const uint32_t bits = f32_to_bf16_bits(sc);
-          reinterpret_cast<uint16_t*>(scores)[(int64_t)qi * ld + s_idx] = (uint16_t)bits;
+          reinterpret_cast<uint16_t*>(scores)[(int64_t)wq * ld + s_idx] = (uint16_t)bits;
           if (hist) atomicAdd(sh + score_bin16(bits), 1u);
         } else {
-          reinterpret_cast<float*>(scores)[(int64_t)qi * ld + s_idx] = sc;
+          reinterpret_cast<float*>(scores)[(int64_t)wq * ld + s_idx] = sc;
           if (hist) atomicAdd(sh + score_bin(sc), 1u);
         }
       }
@@ -372,40 +451,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
 
 // ---- host side ----------------------------------------------------------------
 
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(p);
-  }
-  return fn;
-}
-
-bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
-  EncodeFn f = encode_fn();
-  if (!f) return false;
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = f(map, dt, (cuuint32_t)rank, const_cast<void*>(base), (const cuuint64_t*)dims,
-                 (const cuuint64_t*)strides_bytes, (const cuuint32_t*)box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool index_scores_tc_supported(const csa_params& p, int64_t k_cap, const void* q_idx, const uint8_t* q_sf,
                                const void* k_idx, const uint8_t* k_sf) {
   if (p.idx_fmt != CSA_IDX_MXFP4 || p.n_idx_heads != kHeads || p.idx_dim != 128) return false;
   if (k_cap % 4 != 0) return false;  // scale rows must start 16-byte aligned for TMA
-  return encode_fn() != nullptr;
+  return tensor_maps_available();
 }
 
 cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const uint8_t* q_sf, const float* w,
@@ -413,6 +465,10 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
                                    const int32_t* q_pos0, int T, void* scores, int ld, uint32_t* hist,
                                    int n_max, int32_t* err, cudaStream_t st) {
   const int nq = p.B * T;
+  // prefill (more than 4 queries per sequence): query pairs, 128-entry stages
+  const bool prefill = T > 4;
+  const int qn = prefill ? kPair : 1;
+  const int stage_keys = prefill ? kTileM : kStageKeys;
   CUtensorMap tk, tq, tsk, tsq;
   const uint64_t key_rows = (uint64_t)p.B * (uint64_t)k_cap;
   {
@@ -421,42 +477,46 @@ cudaError_t launch_index_scores_tc(const csa_params& p, const void* q_idx, const
     uint64_t dims[3] = {kRowBytes, key_rows / 4, 4};
     uint64_t str[2] = {4 * kRowBytes, kRowBytes};
     uint32_t box[3] = {kRowBytes, kTileM / 4, 4};
-    if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
   {
     uint64_t dims[2] = {kRowBytes, (uint64_t)nq * kHeads};
     uint64_t str[1] = {kRowBytes};
-    uint32_t box[2] = {kRowBytes, kHeads};
-    if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+    uint32_t box[2] = {kRowBytes, (uint32_t)(qn * kHeads)};
+    if (!encode_tensor_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_idx, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
   }
   {
     uint64_t dims[1] = {key_rows};
     uint64_t str[1] = {4};
-    uint32_t box[1] = {kStageKeys};
-    if (!make_map(&tsk, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, k_sf, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    uint32_t box[1] = {(uint32_t)stage_keys};
+    if (!encode_tensor_map(&tsk, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, k_sf, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
   {
     uint64_t dims[1] = {(uint64_t)nq * kHeads};
     uint64_t str[1] = {4};
-    uint32_t box[1] = {kHeads};
-    if (!make_map(&tsq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, q_sf, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    uint32_t box[1] = {(uint32_t)(qn * kHeads)};
+    if (!encode_tensor_map(&tsq, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, q_sf, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int tpq = (n_max + kStageKeys - 1) / kStageKeys;
-  const int64_t tiles = (int64_t)nq * tpq;
-  const int grid = (int)(tiles < sms ? tiles : sms);
+  const int sms = sm_count();
+  int64_t units;
+  if (prefill) {
+    units = (int64_t)p.B * ((T + kPair - 1) / kPair);  // query pairs
+  } else {
+    const int tpq = (n_max + kStageKeys - 1) / kStageKeys;
+    units = (int64_t)nq * tpq;
+  }
+  const int grid = (int)(units < sms ? units : sms);
   if (grid == 0) return cudaSuccess;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(index_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kfn = prefill ? index_scores_tc<true> : index_scores_tc<false>;
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(kfn), smem);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(index_scores_tc, dim3(grid), dim3(kThreadsTc), smem, st, tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap,
-                 nq, n_max, scores, ld, p.score_fmt == CSA_SCORE_BF16 ? 1 : 0, hist, err);
+  e = launch_pdl(kfn, dim3(grid), dim3(kThreadsTc), smem, st, tk, tq, tsk, tsq, w, q_pos0, T, p.m, k_cap, nq,
+                 n_max, scores, ld, p.score_fmt == CSA_SCORE_BF16 ? 1 : 0, hist, err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

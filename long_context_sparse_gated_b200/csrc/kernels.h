@@ -1,6 +1,7 @@
 // Internal launchers of libcsa (not part of the public ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -12,6 +13,18 @@ namespace csa {
 // Message returned by csa_last_error_string() on this host thread (a string
 // with static storage duration).
 void set_last_error(const char* msg);
+
+// Host-side work done once (host_cache.cu).  Id of the calling thread's
+// current context (0 if none); SM count of the current device; raise a
+// kernel's dynamic shared-memory limit once per device and context; encode
+// a TMA tensor map (no multicast, L2 256-byte promotion, zero fill), reusing
+// a recent identical encode of this host thread.
+unsigned long long current_ctx_id();
+int sm_count();
+cudaError_t set_max_smem(const void* kernel, size_t bytes);
+bool tensor_maps_available();
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw);
 
 // Launch with programmatic stream serialisation (see pdl_wait in
 // common.cuh): the kernel may begin while its predecessor on the stream

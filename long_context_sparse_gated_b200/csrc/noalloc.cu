@@ -49,31 +49,6 @@ struct ScratchSlot {
 ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
-
-// Unique id of the calling thread's current context (0 if unavailable).
-unsigned long long current_ctx_id() {
-  static CtxGetCurrentFn get_cur = nullptr;
-  static CtxGetIdFn get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<CtxGetIdFn>(p);
-  });
-  CUcontext ctx = nullptr;
-  unsigned long long id = 0;
-  if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
-  return 0;
-}
-
 csa_status scratch_for_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -87,7 +62,7 @@ csa_status scratch_for_current_device(void** out) {
   }
   // id of the current context (0 before the runtime has made one current:
   // the lookup below then makes it, and the next call looks up once more)
-  const unsigned long long ctx = current_ctx_id();
+  const unsigned long long ctx = csa::current_ctx_id();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   ScratchSlot& slot = g_scratch[dev];
   if (!slot.addr || slot.ctx_id != ctx) {

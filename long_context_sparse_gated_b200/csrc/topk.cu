@@ -643,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_staged(const void* __restric
 
 template <class K>
 cudaError_t set_smem(K kernel, size_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return set_max_smem(reinterpret_cast<const void*>(kernel), bytes);
 }
 
 template <bool kB16>

@@ -82,3 +82,22 @@ def test_tc_prefill_many_queries():
     for (b, tq), sc in scores.items():
         n_t = len(sc)
         np.testing.assert_array_equal(g[tq, :n_t].astype(np.float64), sc)
+
+
+@pytest.mark.parametrize("score_fmt", ["f32", "bf16"])
+def test_tc_prefill_query_pairs(score_fmt):
+    """Prefill shape (T > 4): the scorer pairs consecutive queries of one
+    sequence into one N=128 MMA.  Two sequences (pairs never cross them),
+    an odd T (the last pair has one query), queries at the start of a
+    sequence that see no entry yet, ragged rows; scores and top-k sets
+    equal the oracle's exactly."""
+    w = synth.with_score_fmt(synth.config("c4", B=2, L=[6000, 4100], T=301, q_pos0=[0, 3700]), score_fmt)
+    dw = _run_index(w)
+    idx, scores = pipeline.index_topk(w, return_scores=True, score_fmt=score_fmt)
+    if score_fmt == "f32":
+        g = _scores(dw)
+        for (b, tq), sc in scores.items():
+            np.testing.assert_array_equal(g[b * w["T"] + tq, :len(sc)].astype(np.float64), sc)
+    got = dw.idx.cpu().numpy()
+    for (b, tq), ref in idx.items():
+        np.testing.assert_array_equal(got[b, tq], ref, err_msg=f"b={b} tq={tq}")
