@@ -87,9 +87,8 @@ struct __align__(1024) AttnSmem {
                               // after the last tile: the [64 heads][512 dims] output stage
   uint8_t p[kRows * 128];     // P' MN-major: [128 rows][64 heads] FP16, 128B swizzle
   uint8_t q[8][kHg * 128];    // 8 K-chunks: [64 heads][128 B]
-  float scale[kRows];
-  float code_mul[kRows];      // 2^k_j: factor of the row's E4M3 codes in V'
-  float rope_mul[kRows];      // 2^k_j / s_j: factor of its RoPE dims in V'
+  const uint8_t* rowp[2][kRows];  // stored row of each tile slot (null: empty), tiles i and i+1
+  float rsc[2][kRows];            // its scale s_j
   float row_f[kRows];         // tau * log2(e) * c_j  (c_j = s_j 2^-k_j)
   float row_lc[kRows];        // log2 c_j
   float row_ic[kRows];        // 1 / c_j
@@ -99,18 +98,12 @@ struct __align__(1024) AttnSmem {
   float red[kWarps][32];
   float mh[kHg], lh[kHg], alpha[kHg];
   float rope_c[kR / 2], rope_s[kR / 2];  // inverse-RoPE rotation of this query
-  uint64_t bar_q, bar_g, bar_s, bar_o;
+  uint64_t bar_q, bar_s, bar_o;
   uint32_t tmem_base;
   int abort;
   int rescale;
 };
 
-// The raw rows of a tile (128 x 576 B) are staged in V' chunks 4..7 and the
-// P' buffer that follows them; both are free while a tile is gathered.
-constexpr int kStageOff = 4 * kRows * 128;
-static_assert(offsetof(AttnSmem, p) == sizeof(((AttnSmem*)0)->v), "P' must follow V'");
-static_assert(kStageOff + kRows * kRowBytes <= (int)(sizeof(((AttnSmem*)0)->v) + sizeof(((AttnSmem*)0)->p)),
-              "staging area");
 
 __device__ __forceinline__ uint32_t sw128(int row, int chunk16) {
   return (uint32_t)(row * 128 + ((chunk16 ^ (row & 7)) << 4));
@@ -280,7 +273,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
 
   if (issuer) {
     sm100::mbar_init(&S.bar_q, 1);
-    sm100::mbar_init(&S.bar_g, 1);
     sm100::mbar_init(&S.bar_s, 1);
     sm100::mbar_init(&S.bar_o, 1);
     S.abort = 0;
@@ -339,43 +331,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   // Row of this thread (wt < kRows) in the current tile, resolved one tile
   // ahead: while tile i is computed, tile i+1's rows are resolved, their
   // scales loaded and their bytes prefetched into L2.
-  int my_src = 0;
-  int64_t my_off = -1;
-  float my_sc = 1.f;
-  if (wt < kRows && n_tiles > 0) {
-    my_src = resolve_slot<kDense>(sb + wt, se, own_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap, err, &my_off);
-    if (my_src == 1) my_sc = cache_scale[my_off];
-    if (my_src == 2) my_sc = win_scale[my_off];
-  }
+  auto resolve_to = [&](int buf, int slot) {
+    int64_t off = -1;
+    const int src = resolve_slot<kDense>(slot, se, own_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap, err, &off);
+    const uint8_t* rp = nullptr;
+    float sc = 1.f;
+    if (src == 1) { rp = cache_rows + off * kRowBytes; sc = cache_scale[off]; }
+    if (src == 2) { rp = win_rows + off * kRowBytes; sc = win_scale[off]; }
+    S.rowp[buf][wt] = rp;
+    S.rsc[buf][wt] = sc;
+    return rp;
+  };
+  if (wt < kRows && n_tiles > 0) resolve_to(0, sb + wt);
 
   // Control flow is uniform across the CTA (every __syncthreads is reached
   // by all threads); a failed bounded wait only raises the abort flag,
   // after which every later wait returns at once and no MMA is issued.
   for (int i = 0; i < n_tiles; ++i) {
     const int tb = sb + i * kRows;
-    if (i > 0) sm100::mbar_wait(&S.bar_o, (i - 1) & 1, abort);  // V' and P' buffers free
+    if (i == 0) __syncthreads();  // tile 0's row pointers visible
     if (wt == 0) S.rescale = 0;
-    const int n_copy = __syncthreads_count(my_src != 0);
-    if (issuer) sm100::mbar_arrive_expect_tx(&S.bar_g, (uint32_t)(n_copy * kRowBytes));
-    __syncthreads();
-    // -- gather: one bulk copy per non-empty row (rows and the staging area
-    //    are 16-byte aligned, 576 = 36 x 16 bytes)
-    uint8_t* stg = &S.v[0][0] + kStageOff;
-    if (my_src) {
-      const uint8_t* src = (my_src == 2 ? win_rows : cache_rows) + my_off * kRowBytes;
-      sm100::bulk_load(stg + wt * kRowBytes, src, kRowBytes, &S.bar_g);
-    }
-    if (wt < kRows) {
-      float sc = my_sc;
-      int live = my_src != 0;
-      if (!(sc >= 0x1p-90f) || !(sc <= 0x1p90f)) {  // outside the supported scale range
-        if (my_src) raise_err(err, CSA_DEV_ERR_RANGE);
-        live = 0;  // the row is dropped (zeroed below)
-        sc = 1.f;
-      }
-      S.live[wt] = live;
-      S.scale[wt] = sc;
-    }
+    // -- gather: this thread's share of the tile, row r (8-row block `warp`),
+    //    16-byte chunks 4k + lane%4 (k < 7: E4M3 codes of K-chunk k; k = 7, 8:
+    //    RoPE dims), straight from global memory into registers.  The loads
+    //    are issued before the wait for the previous tile's O MMA, so they
+    //    overlap it; the rows were prefetched into L2 during that tile.
+    const int r = 8 * warp + (lane >> 2);
+    const uint8_t* rp = S.rowp[i & 1][r];
+    float sc = S.rsc[i & 1][r];
+    uint4 raw[kLoads];
+#pragma unroll
+    for (int k = 0; k < kLoads; ++k)
+      raw[k] = rp ? __ldg(reinterpret_cast<const uint4*>(rp + (4 * k + (lane & 3)) * 16)) : make_uint4(0, 0, 0, 0);
+    if (i > 0) sm100::mbar_wait(&S.bar_o, (i - 1) & 1, abort);  // V' and P' buffers free
     if (i == 0) {
       // each head's largest BF16 query magnitude (converted after the
       // barrier).  Word e of the query tile is head ((e >> 3) & 63): this
@@ -389,38 +377,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       for (int o = 1; o < 8; o <<= 1) ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, o));
       if ((lane & 7) == 0) atomicMax(&S.qamax[wt >> 3], ma << 16);
     }
-    // Conversion work: (8-row block, group of four 16-byte chunks) pairs,
-    // one pair per warp instruction, lane = 4 x row-in-block + chunk-in-group:
-    // both the staging reads and the swizzled V' stores then spread a warp's
-    // 32 x 16 bytes over all banks.
-    sm100::mbar_wait(&S.bar_g, i & 1, abort);
-    if (wt < kRows) {
-      // row prep: the row's largest RoPE magnitude, its shift k_j and the
-      // factors of its codes, RoPE dims, logits and denominator terms
-      const uint4* rp = reinterpret_cast<const uint4*>(stg + wt * kRowBytes + kNope);
-      uint32_t rb = 0;
-#pragma unroll
-      for (int x = 0; x < 2 * kR / 16; ++x) rb = max(rb, bf16x8_amax_bits(rp[x]));
-      const float sc = S.scale[wt];
+    // -- row factors (the four lanes of row r agree): the row's largest RoPE
+    //    magnitude, its shift k_j, the factors of its codes and RoPE dims, and
+    //    for the softmax those of its logits and denominator terms
+    bool live = rp != nullptr;
+    if (!(sc >= 0x1p-90f) || !(sc <= 0x1p90f)) {  // outside the supported scale range
+      if (live) raise_err(err, CSA_DEV_ERR_RANGE);
+      live = false;  // the row is dropped (zeros)
+      sc = 1.f;
+    }
+    float code_mul, rope_mul;
+    {
+      uint32_t rb = max(bf16x8_amax_bits(raw[kLoads - 2]), bf16x8_amax_bits(raw[kLoads - 1]));
+      rb = max(rb, __shfl_xor_sync(0xffffffffu, rb, 1));
+      rb = max(rb, __shfl_xor_sync(0xffffffffu, rb, 2));
       const int kr = row_shift(sc, rb);
       const float cj = ldexpf(sc, -kr);
-      const bool live = S.live[wt] != 0;
-      S.code_mul[wt] = kr >= -24 ? __uint_as_float((uint32_t)(127 + kr) << 23) : 0.f;
-      S.rope_mul[wt] = ldexpf(1.f / sc, kr);
-      S.row_f[wt] = live ? tau * kLog2e * cj : 0.f;
-      S.row_lc[wt] = log2f(cj);
-      S.row_ic[wt] = 1.f / cj;
+      code_mul = kr >= -24 ? __uint_as_float((uint32_t)(127 + kr) << 23) : 0.f;
+      rope_mul = ldexpf(1.f / sc, kr);
+      if ((lane & 3) == 0) {
+        S.live[r] = live;
+        S.row_f[r] = live ? tau * kLog2e * cj : 0.f;
+        S.row_lc[r] = log2f(cj);
+        S.row_ic[r] = 1.f / cj;
+      }
     }
-    // Pair k of this warp: chunk group k (compile-time: groups 0-6 are E4M3
-    // codes, 7-8 RoPE dims) of 8-row block `warp`.
-    uint4 raw[kLoads];
-#pragma unroll
-    for (int k = 0; k < kLoads; ++k) {
-      const int r = 8 * warp + (lane >> 2), c = 4 * k + (lane & 3);
-      raw[k] = *reinterpret_cast<const uint4*>(stg + r * kRowBytes + c * 16);
-    }
-    __syncthreads();  // staging area read by all; row factors, live flags, query amax visible
     if (i == 0) {
+      __syncthreads();  // query amax complete
       // each head's power-of-two range factor 2^e_h: Q'_h = Q_h 2^-e_h has
       // its largest magnitude in [2^14, 2^15)
       auto head_exp = [&](int h) {
@@ -433,21 +416,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
 #pragma unroll 4
       for (int e = wt; e < 8 * kHg * 128 / 16; e += kThreads) qv[e] = bf16x8_scale_to_f16(qv[e], qia);
     }
-    // -- convert + store V' (empty and dropped rows as zeros: the staging
-    //    area holds stale bytes there)
+    // -- convert + store V' (empty and dropped rows as zeros)
 #pragma unroll
     for (int k = 0; k < kLoads; ++k) {
-      const int r = 8 * warp + (lane >> 2), c = 4 * k + (lane & 3);
-      const bool live = S.live[r] != 0;
+      const int c = 4 * k + (lane & 3);
       if (k < kNope / 64) {
         // dims 16c .. 16c+15 -> K-chunk (16c)/64, 16-byte slots 2(c%4), 2(c%4)+1;
         // codes times 2^k (exact down to 2^-24)
         uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
         if (live) {
           e4m3x16_to_f16(raw[k], lo, hi);
-          const float cm = S.code_mul[r];
-          if (cm != 1.f) {
-            const __half2 f = __float2half2_rn(cm);
+          if (code_mul != 1.f) {
+            const __half2 f = __float2half2_rn(code_mul);
             __half2* ph = reinterpret_cast<__half2*>(&lo);
             __half2* qh = reinterpret_cast<__half2*>(&hi);
 #pragma unroll
@@ -462,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
         // c-28, read by both MMAs), lo at the same place of the P' buffer
         // (free until the softmax; read by the S MMA only)
         uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
-        if (live) bf16x8_scale_to_f16_hilo(raw[k], S.rope_mul[r], hi, lo);
+        if (live) bf16x8_scale_to_f16_hilo(raw[k], rope_mul, hi, lo);
         *reinterpret_cast<uint4*>(S.v[7] + sw128(r, c - kNope / 16)) = hi;
         *reinterpret_cast<uint4*>(S.p + sw128(r, c - kNope / 16)) = lo;
       }
@@ -487,15 +467,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       }
     }
     // -- next tile: resolve, scale load and L2 prefetch while this one runs
-    int nx_src = 0;
-    int64_t nx_off = -1;
-    float nx_sc = 1.f;
     if (wt < kRows && i + 1 < n_tiles) {
-      nx_src = resolve_slot<kDense>(tb + kRows + wt, se, own_sel, t, n_t, W, bs, qi, idx, topk, cache_cap,
-                                    win_cap, err, &nx_off);
-      if (nx_src) sm100::bulk_prefetch_l2((nx_src == 2 ? win_rows : cache_rows) + nx_off * kRowBytes, kRowBytes);
-      if (nx_src == 1) nx_sc = cache_scale[nx_off];
-      if (nx_src == 2) nx_sc = win_scale[nx_off];
+      const uint8_t* nx = resolve_to((i + 1) & 1, tb + kRows + wt);
+      if (nx) sm100::bulk_prefetch_l2(nx, kRowBytes);
     }
     sm100::mbar_wait(&S.bar_s, i & 1, abort);
     sm100::tc_fence_after();
@@ -607,9 +581,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
         sm100::tc_commit(&S.bar_o);
       }
     }
-    my_src = nx_src;
-    my_off = nx_off;
-    my_sc = nx_sc;
   }
 
   pdl_trigger();
@@ -793,27 +764,11 @@ __global__ void __launch_bounds__(256) attn_merge_f32(const float* __restrict__ 
   dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(p);
-  }
-  return fn;
-}
-
 }  // namespace
 
 bool attn_tc_supported(const csa_params& p) {
   return p.kv_fmt == CSA_KV_FP8_BF16 && p.act_fmt == CSA_ACT_BF16 && p.d == kD && p.r == kR &&
-         p.n_heads % kHg == 0 && encode_fn() != nullptr;
+         p.n_heads % kHg == 0 && tensor_maps_available();
 }
 
 // Rows per split, a function of the call's parameters and T only -- never
@@ -841,13 +796,10 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
   const int nq = p.B * T;
   CUtensorMap tq;
   {
-    cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)nq * p.n_heads};
-    cuuint64_t str[1] = {(cuuint64_t)kD * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kHg};
-    cuuint32_t es[2] = {1, 1};
-    if (encode_fn()(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, str, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    uint64_t dims[2] = {(uint64_t)kD, (uint64_t)nq * p.n_heads};
+    uint64_t str[1] = {(uint64_t)kD * 2};
+    uint32_t box[2] = {64, (uint32_t)kHg};
+    if (!encode_tensor_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   const int total = n_sel + p.window;
@@ -860,7 +812,7 @@ cudaError_t launch_attn_tc(const csa_params& p, const void* q, const csa_kv& cac
   float* ws_ml = ws ? ws + n_part * p.d : nullptr;
   const size_t smem = attn_tc_smem_bytes();
   auto kfn = dense ? attn_tc<true> : attn_tc<false>;
-  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(kfn), smem);
   if (e != cudaSuccess) return e;
   dim3 grid(nq, n_splits, nhg);
   e = launch_pdl(kfn, grid, dim3(kThreads), smem, st, tq, reinterpret_cast<const uint8_t*>(cache.rows), cache.scale,
