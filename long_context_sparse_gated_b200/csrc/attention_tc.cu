@@ -481,6 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       uint32_t a[16];
       sm100::tmem_ld_x16(s_col + ((uint32_t)(quad * 32) << 16) + kHPart * part, a);
       sm100::tmem_ld_wait();
+      sm100::tmem_pin16(a);
       const bool valid = S.live[j] != 0;
       const float f = S.row_f[j];
       const float lc = S.row_lc[j];
@@ -530,6 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
         const uint32_t ta = o_col + 64 * blk + ((uint32_t)(quad * 32) << 16) + kHPart * part;
         sm100::tmem_ld_x16(ta, r16);
         sm100::tmem_ld_wait();
+        sm100::tmem_pin16(r16);
 #pragma unroll
         for (int c = 0; c < 16; ++c) r16[c] = __float_as_uint(__uint_as_float(r16[c]) * S.alpha[kHPart * part + c]);
         sm100::tmem_st_x16(ta, r16);
@@ -621,6 +623,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
       for (int x = 0; x < 2; ++x)
         sm100::tmem_ld_x16(o_col + 64 * (b2 + x) + ((uint32_t)(quad * 32) << 16) + kHPart * part, rr[x]);
       sm100::tmem_ld_wait();
+      sm100::tmem_pin16(rr[0]);
+      sm100::tmem_pin16(rr[1]);
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const int blk = b2 + x;

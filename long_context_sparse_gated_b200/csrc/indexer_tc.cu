@@ -406,21 +406,31 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       // after an abort every wait returns at once and no work is done
       if (!__shfl_sync(0xffffffffu, ok, 0)) continue;
       sm100::tc_fence_after();
+      // the 64 head columns in two halves: the second half's load is in
+      // flight while the first half is summed
       uint32_t d[64];
+      auto grp = [&](int g) -> uint32_t(&)[16] { return *reinterpret_cast<uint32_t(*)[16]>(d + 16 * g); };
       const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + (acc * kTiles + eg) * kHeads;
-      sm100::tmem_ld_x16(base + 0, *reinterpret_cast<uint32_t(*)[16]>(d + 0));
-      sm100::tmem_ld_x16(base + 16, *reinterpret_cast<uint32_t(*)[16]>(d + 16));
-      sm100::tmem_ld_x16(base + 32, *reinterpret_cast<uint32_t(*)[16]>(d + 32));
-      sm100::tmem_ld_x16(base + 48, *reinterpret_cast<uint32_t(*)[16]>(d + 48));
+      sm100::tmem_ld_x16(base + 0, grp(0));
+      sm100::tmem_ld_x16(base + 16, grp(1));
       sm100::tmem_ld_wait();
-      sm100::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(&S.tempty[acc]);
+      sm100::tmem_pin16(grp(0));
+      sm100::tmem_pin16(grp(1));
+      sm100::tmem_ld_x16(base + 32, grp(2));
+      sm100::tmem_ld_x16(base + 48, grp(3));
       // four independent partial sums (every partial sum of these
       // scores is exact, so the grouping does not change the result)
       float p4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) p4[h & 3] = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), p4[h & 3]);
+      for (int h = 0; h < kHeads / 2; ++h) p4[h & 3] = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), p4[h & 3]);
+      sm100::tmem_ld_wait();
+      sm100::tmem_pin16(grp(2));
+      sm100::tmem_pin16(grp(3));
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&S.tempty[acc]);
+#pragma unroll
+      for (int h = kHeads / 2; h < kHeads; ++h) p4[h & 3] = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), p4[h & 3]);
       const float sc = (p4[0] + p4[1]) + (p4[2] + p4[3]);
       const int s_idx = wk.j * M::kKeys + (kPrefill ? 0 : eg * kTileM) + key_in_tile;
       if (s_idx < n_t) {

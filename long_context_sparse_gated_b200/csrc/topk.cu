@@ -646,11 +646,152 @@ cudaError_t set_smem(K kernel, size_t bytes) {
   return set_max_smem(reinterpret_cast<const void*>(kernel), bytes);
 }
 
+// ---- no-histogram mode, rows of up to kCap entries: 256 threads per query ----
+//
+// Many queries with short rows (prefill): one 8-warp CTA per query, several
+// CTAs per SM.  The row's keys are staged in shared memory (sized by the
+// row bound), the radix select takes 8-bit passes over them, and the
+// ordered compaction gives each warp a contiguous run of entries walked in
+// 32-entry slabs (lane-strided, so shared-memory reads are conflict-free;
+// ballots give in-slab ranks): one pass counts the run's keys equal to the
+// threshold, one counts its selected entries, one writes their indices.
+constexpr int kRowThreads = 256;
+constexpr int kRowWarps = kRowThreads / 32;
+
+// exclusive scan of one int per warp (lane 0's value counts) over the
+// kRowWarps warps; every thread gets its warp's prefix, *total the sum.
+__device__ __forceinline__ int warp_prefix(int v, int* tmp, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) tmp[wid] = v;
+  __syncthreads();
+  int pre = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kRowWarps; ++w) {
+    const int x = tmp[w];
+    pre += w < wid ? x : 0;
+    tot += x;
+  }
+  __syncthreads();
+  *total = tot;
+  return pre;
+}
+
+template <bool kB16>
+__global__ void __launch_bounds__(kRowThreads) topk_rows(const void* __restrict__ scores, int ld, int n_max,
+                                                         const int32_t* __restrict__ q_pos0, int T, int m, int k,
+                                                         int32_t* __restrict__ out_idx) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(smem_raw);
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t sel[2];
+  __shared__ int tmp[kRowWarps];
+  pdl_wait();
+  pdl_trigger();
+  const int qi = blockIdx.x;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int n_t = visible_entries(q_pos0, T, m, qi, n_max);
+  const void* row = score_row<kB16>(scores, qi, ld);
+  int32_t* out = out_idx + (int64_t)qi * k;
+  if (n_t <= k) {
+    for (int i = threadIdx.x; i < k; i += kRowThreads) out[i] = i < n_t ? i : -1;
+    return;
+  }
+  // stage the keys (coalesced 16-byte loads: 4 fp32 or 8 BF16 scores)
+  constexpr int kPer = kB16 ? 8 : 4;
+  for (int s = kPer * threadIdx.x; s < n_t; s += kPer * kRowThreads) {
+    uint32_t kk[kPer];
+    if (kB16) {
+      const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(row) + s);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        kk[2 * j] = score_key16(w[j]);
+        kk[2 * j + 1] = score_key16(w[j] >> 16);
+      }
+    } else {
+      const float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row) + s);
+      kk[0] = score_key(v.x);
+      kk[1] = score_key(v.y);
+      kk[2] = score_key(v.z);
+      kk[3] = score_key(v.w);
+    }
+#pragma unroll
+    for (int e = 0; e < kPer; ++e)
+      if (s + e < n_t) ckey[s + e] = kk[e];
+  }
+  // radix select: the key thr of the k-th largest and how many keys equal
+  // to it are taken (`need`)
+  uint32_t prefix = 0, mask = 0;
+  int need = k;
+  for (int shift = ScoreKeys<kB16>::kBits - 8; shift >= 0; shift -= 8) {
+    hist[threadIdx.x] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_t; i += kRowThreads) {
+      const uint32_t key = ckey[i];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    if (wid == 0) find_bin256(hist, (uint32_t)need, sel);
+    __syncthreads();
+    prefix |= sel[0] << shift;
+    mask |= 0xFFu << shift;
+    need -= (int)sel[1];
+  }
+  const uint32_t thr = prefix;
+  // ordered compaction over warp runs of whole 32-entry slabs
+  const int slabs = (n_t + 31) / 32;
+  const int per_warp = (slabs + kRowWarps - 1) / kRowWarps;
+  const int s0 = wid * per_warp, s1 = min(slabs, s0 + per_warp);
+  const unsigned below = (1u << lane) - 1u;
+  int n_eq = 0;
+  for (int sl = s0; sl < s1; ++sl) {
+    const int i = 32 * sl + lane;
+    n_eq += __popc(__ballot_sync(0xffffffffu, i < n_t && ckey[i] == thr));
+  }
+  int tot;
+  const int eq0 = warp_prefix(n_eq, tmp, &tot);
+  int n_sel = 0;
+  {
+    int er = eq0;
+    for (int sl = s0; sl < s1; ++sl) {
+      const int i = 32 * sl + lane;
+      const uint32_t key = i < n_t ? ckey[i] : 0u;
+      const unsigned eq = __ballot_sync(0xffffffffu, i < n_t && key == thr);
+      const unsigned gt = __ballot_sync(0xffffffffu, i < n_t && key > thr);
+      // equal keys of this slab ranked er, er+1, ... in index order
+      const int avail = max(0, min(need - er, 32));
+      n_sel += __popc(gt) + min(__popc(eq), avail);
+      er += __popc(eq);
+    }
+  }
+  const int pos0 = warp_prefix(n_sel, tmp, &tot);
+  {
+    int er = eq0, pos = pos0;
+    for (int sl = s0; sl < s1; ++sl) {
+      const int i = 32 * sl + lane;
+      const uint32_t key = i < n_t ? ckey[i] : 0u;
+      const bool is_eq = i < n_t && key == thr;
+      const unsigned eq = __ballot_sync(0xffffffffu, is_eq);
+      const bool take = (i < n_t && key > thr) || (is_eq && er + __popc(eq & below) < need);
+      const unsigned tk = __ballot_sync(0xffffffffu, take);
+      if (take) out[pos + __popc(tk & below)] = i;
+      pos += __popc(tk);
+      er += __popc(eq);
+    }
+  }
+}
+
 template <bool kB16>
 cudaError_t launch_topk_t(const csa_params& p, const void* scores, int ld, int n_max, const uint32_t* hist,
                           void* extra, const int32_t* q_pos0, int T, int32_t* out_idx, cudaStream_t st) {
   const int nq = p.B * T;
   cudaError_t e;
+  if (!hist && n_max <= kCap) {
+    const size_t smem = (size_t)((n_max + 3) & ~3) * 4;
+    if ((e = set_smem(topk_rows<kB16>, smem)) != cudaSuccess) return e;
+    return launch_pdl(topk_rows<kB16>, dim3(nq), dim3(kRowThreads), smem, st, scores, ld, n_max, q_pos0, T, p.m,
+                      p.topk, out_idx);
+  }
   if (!hist) {
     const size_t smem = sizeof(StageSmem) > sizeof(BitSmem) ? sizeof(StageSmem) : sizeof(BitSmem);
     if ((e = set_smem(topk_staged<kB16>, smem)) != cudaSuccess) return e;

@@ -102,3 +102,15 @@ def test_topk_staged_selector(fmt):
 def test_topk_prefill_rows(fmt):
     w = synth.with_score_fmt(synth.config("c4", B=1, L=4096, T=200, q_pos0=3000), fmt)
     _check(w, _run(w))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_topk_rows_heavy_ties(fmt):
+    """No-histogram mode with every score of a row equal (all index keys
+    the same): the row selector keeps the k lowest indices."""
+    w = synth.with_score_fmt(synth.with_index_heads(synth.config("c1", B=2, L=8192), 32), fmt)
+    w["k_idx"][...] = w["k_idx"][:, :1]
+    w["k_idx_sf"][...] = w["k_idx_sf"][:, :1]
+    dw = _run(w)
+    for b in range(2):
+        np.testing.assert_array_equal(dw.idx[b, 0].cpu().numpy(), np.arange(512))
