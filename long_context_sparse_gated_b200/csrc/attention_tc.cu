@@ -649,16 +649,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
         }
       }
     }
+    sm100::fence_proxy_async_smem();
     __syncthreads();
-    // 64 rows of 1 KB (BF16) or 2 KB (fp32), 16-byte words
-    if (single) {
-      uint4* dst0 = reinterpret_cast<uint4*>(out + ((int64_t)qi * n_heads + h0) * kD);
-#pragma unroll 4
-      for (int u = wt; u < kHg * kD / 8; u += kThreads) dst0[u] = reinterpret_cast<const uint4*>(stage)[u];
-    } else {
-      uint4* dst0 = reinterpret_cast<uint4*>(ws_o + (((int64_t)qi * n_splits + split) * n_heads + h0) * kD);
-#pragma unroll 4
-      for (int u = wt; u < kHg * kD / 4; u += kThreads) dst0[u] = reinterpret_cast<const uint4*>(stage32)[u];
+    // the 64 x 512 block is contiguous in the output (64 rows of 1 KB BF16)
+    // and in the split partials (2 KB fp32 rows): one bulk store
+    if (issuer) {
+      if (single)
+        sm100::bulk_store(out + ((int64_t)qi * n_heads + h0) * kD, stage, kHg * kD * 2);
+      else
+        sm100::bulk_store(ws_o + (((int64_t)qi * n_splits + split) * n_heads + h0) * kD, stage32, kHg * kD * 4);
+      sm100::bulk_commit();
+      sm100::bulk_wait_read();  // shared memory read before the CTA exits
     }
     if (!single && wt < kHg) {
       const int64_t base = ((int64_t)qi * n_splits + split) * n_heads + h0 + wt;
