@@ -49,7 +49,7 @@
 // dropped with CSA_DEV_ERR_RANGE.
 //
 // 16 warps (four per TMEM lane quadrant, 16 heads each) gather, convert
-// (warp w: row block w), run the softmax and the epilogue; thread 0 also
+// (warp w: row block w), run the softmax and the epilogue; thread 128 also
 // issues the query TMA and the MMAs between block barriers.  Every wait is
 // bounded (CSA_DEV_ERR_TIMEOUT).
 #include <cuda.h>
@@ -88,7 +88,7 @@ struct __align__(1024) AttnSmem {
   uint8_t p[kRows * 128];     // P' MN-major: [128 rows][64 heads] FP16, 128B swizzle
   uint8_t q[8][kHg * 128];    // 8 K-chunks: [64 heads][128 B]
   const uint8_t* rowp[2][kRows];  // stored row of each tile slot (null: empty), tiles i and i+1
-  float rsc[2][kRows];            // its scale s_j
+  const float* rscp[2][kRows];    // its scale s_j
   float row_f[kRows];         // tau * log2(e) * c_j  (c_j = s_j 2^-k_j)
   float row_lc[kRows];        // log2 c_j
   float row_ic[kRows];        // 1 / c_j
@@ -224,12 +224,21 @@ __device__ __forceinline__ float warp_transpose_reduce16(float (&v)[16]) {
   return kMax ? fmaxf(v[0], o) : v[0] + o;
 }
 
-// Row of candidate slot `slot` (< se) of query t: src 1 = cache row, 2 =
-// window ring row, 0 = empty; *off = element row index into that array.
+// The selected entry held by candidate slot `slot` of query qi (sparse
+// mode, slot < n_sel < se), loaded ahead of its use; -1 otherwise.
 template <bool kDense>
-__device__ __forceinline__ int resolve_slot(int slot, int se, int n_sel, int64_t t, int64_t n_t, int W, int bs, int qi,
-                                            const int32_t* __restrict__ idx, int topk, int64_t cache_cap,
-                                            int64_t win_cap, int32_t* err, int64_t* off) {
+__device__ __forceinline__ int slot_entry(int slot, int se, int n_sel, int qi, const int32_t* __restrict__ idx,
+                                          int topk) {
+  if (kDense || slot >= se || slot >= n_sel) return -1;
+  return __ldg(idx + (int64_t)qi * topk + slot);
+}
+
+// Row of candidate slot `slot` (< se) of query t, given its entry e from
+// slot_entry: src 1 = cache row, 2 = window ring row, 0 = empty; *off =
+// element row index into that array.
+template <bool kDense>
+__device__ __forceinline__ int resolve_slot(int slot, int e, int se, int n_sel, int64_t t, int64_t n_t, int W, int bs,
+                                            int64_t cache_cap, int64_t win_cap, int32_t* err, int64_t* off) {
   int src = 0;
   int64_t row = 0;
   if (slot < se) {
@@ -237,7 +246,6 @@ __device__ __forceinline__ int resolve_slot(int slot, int se, int n_sel, int64_t
       if (kDense) {
         if (slot < n_t && slot < cache_cap) { src = 1; row = slot; }
       } else {
-        const int e = idx[(int64_t)qi * topk + slot];
         if (e >= 0 && e < n_t && e < cache_cap) { src = 1; row = e; }
         else if (e != -1) raise_err(err, CSA_DEV_ERR_INDEX);
       }
@@ -269,7 +277,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   const int bs = qi / T, tq = qi % T;
   const int h0 = hg * kHg;
   volatile int* abort = &S.abort;
-  const bool issuer = threadIdx.x == 0;
+  // MMA / TMA issuer: warp 4 resolves no rows and updates no head sums, so
+  // its lane 0 is free when a tile's operands are ready
+  const bool issuer = threadIdx.x == 128;
 
   if (issuer) {
     sm100::mbar_init(&S.bar_q, 1);
@@ -331,18 +341,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
   // Row of this thread (wt < kRows) in the current tile, resolved one tile
   // ahead: while tile i is computed, tile i+1's rows are resolved, their
   // scales loaded and their bytes prefetched into L2.
-  auto resolve_to = [&](int buf, int slot) {
+  // the row and scale addresses of a slot (its entry pre-loaded); the
+  // scales are loaded together with the rows' bytes
+  auto resolve_to = [&](int buf, int slot, int e) {
     int64_t off = -1;
-    const int src = resolve_slot<kDense>(slot, se, own_sel, t, n_t, W, bs, qi, idx, topk, cache_cap, win_cap, err, &off);
+    const int src = resolve_slot<kDense>(slot, e, se, own_sel, t, n_t, W, bs, cache_cap, win_cap, err, &off);
     const uint8_t* rp = nullptr;
-    float sc = 1.f;
-    if (src == 1) { rp = cache_rows + off * kRowBytes; sc = cache_scale[off]; }
-    if (src == 2) { rp = win_rows + off * kRowBytes; sc = win_scale[off]; }
+    const float* sp = nullptr;
+    if (src == 1) { rp = cache_rows + off * kRowBytes; sp = cache_scale + off; }
+    if (src == 2) { rp = win_rows + off * kRowBytes; sp = win_scale + off; }
     S.rowp[buf][wt] = rp;
-    S.rsc[buf][wt] = sc;
+    S.rscp[buf][wt] = sp;
     return rp;
   };
-  if (wt < kRows && n_tiles > 0) resolve_to(0, sb + wt);
+  if (wt < kRows && n_tiles > 0) resolve_to(0, sb + wt, slot_entry<kDense>(sb + wt, se, own_sel, qi, idx, topk));
 
   // Control flow is uniform across the CTA (every __syncthreads is reached
   // by all threads); a failed bounded wait only raises the abort flag,
@@ -358,11 +370,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     //    overlap it; the rows were prefetched into L2 during that tile.
     const int r = 8 * warp + (lane >> 2);
     const uint8_t* rp = S.rowp[i & 1][r];
-    float sc = S.rsc[i & 1][r];
+    const float* sp = S.rscp[i & 1][r];
     uint4 raw[kLoads];
 #pragma unroll
     for (int k = 0; k < kLoads; ++k)
       raw[k] = rp ? __ldg(reinterpret_cast<const uint4*>(rp + (4 * k + (lane & 3)) * 16)) : make_uint4(0, 0, 0, 0);
+    float sc = sp ? __ldg(sp) : 1.f;
+    // the next tile's selected entries: loaded now, resolved after this
+    // tile's S MMAs are issued
+    const int nx_slot = tb + kRows + wt;
+    const int nx_e = (wt < kRows && i + 1 < n_tiles) ? slot_entry<kDense>(nx_slot, se, own_sel, qi, idx, topk) : -1;
     if (i > 0) sm100::mbar_wait(&S.bar_o, (i - 1) & 1, abort);  // V' and P' buffers free
     if (i == 0) {
       // each head's largest BF16 query magnitude (converted after the
@@ -468,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc(
     }
     // -- next tile: resolve, scale load and L2 prefetch while this one runs
     if (wt < kRows && i + 1 < n_tiles) {
-      const uint8_t* nx = resolve_to((i + 1) & 1, tb + kRows + wt);
+      const uint8_t* nx = resolve_to((i + 1) & 1, nx_slot, nx_e);
       if (nx) sm100::bulk_prefetch_l2(nx, kRowBytes);
     }
     sm100::mbar_wait(&S.bar_s, i & 1, abort);
