@@ -722,6 +722,18 @@ __global__ void __launch_bounds__(256) attn_merge_f32(const float* __restrict__ 
     rope_c[threadIdx.x] = c;
     rope_s[threadIdx.x] = sn;
   }
+  // lane's dims: 4 lane + 128 e (e < 4), so that every float4 load of the
+  // warp reads 512 contiguous bytes; the first four splits' partials are
+  // loaded before their weights are known
+  const float* src0 = ws_o + ((int64_t)qi * n_splits * n_heads + h) * kD + 4 * lane;
+  const int64_t sstride = (int64_t)n_heads * kD;
+  float4 pre[4][4];
+#pragma unroll
+  for (int sp = 0; sp < 4; ++sp)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      pre[sp][e] = sp < own_splits ? __ldg(reinterpret_cast<const float4*>(src0 + sp * sstride + 128 * e))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
   const float sg = sink[h];
   const int64_t ml0 = ((int64_t)qi * n_splits * n_heads + h) * 2;  // split sp at ml0 + 2 sp n_heads
   float m_l = -INFINITY, l_l = 0.f;
@@ -741,13 +753,27 @@ __global__ void __launch_bounds__(256) attn_merge_f32(const float* __restrict__ 
   const float den = expf(sg - M) + warp_sum(part);
   const float inv = den > 0.f ? 1.f / den : 0.f;
   const float a_l = p_l * inv;  // weight of split `lane` (for lane < 32)
-  const int c0 = 16 * lane;
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-  const float* src0 = ws_o + ((int64_t)qi * n_splits * n_heads + h) * kD + c0;
-#pragma unroll 4
-  for (int sp = 0; sp < own_splits; ++sp) {
+  // splits in order; a split of weight zero (empty, or its max far below)
+  // is skipped: its partial may be stale
+  auto add = [&](float a, const float4 (&v)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[4 * e] = fmaf(a, v[e].x, acc[4 * e]);
+      acc[4 * e + 1] = fmaf(a, v[e].y, acc[4 * e + 1]);
+      acc[4 * e + 2] = fmaf(a, v[e].z, acc[4 * e + 2]);
+      acc[4 * e + 3] = fmaf(a, v[e].w, acc[4 * e + 3]);
+    }
+  };
+#pragma unroll
+  for (int sp = 0; sp < 4; ++sp) {
+    const float a = __shfl_sync(0xffffffffu, a_l, sp);
+    if (sp < own_splits && a != 0.f) add(a, pre[sp]);
+  }
+#pragma unroll 2
+  for (int sp = 4; sp < own_splits; ++sp) {
     float a;
     if (sp < 32) {
       a = __shfl_sync(0xffffffffu, a_l, sp);
@@ -756,34 +782,30 @@ __global__ void __launch_bounds__(256) attn_merge_f32(const float* __restrict__ 
       a = ms == -INFINITY ? 0.f : ws_ml[ml0 + (int64_t)2 * sp * n_heads + 1] * expf(ms - M) * inv;
     }
     if (a == 0.f) continue;
-    const float4* src = reinterpret_cast<const float4*>(src0 + (int64_t)sp * n_heads * kD);
+    float4 v[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 v = src[e];
-      acc[4 * e] = fmaf(a, v.x, acc[4 * e]);
-      acc[4 * e + 1] = fmaf(a, v.y, acc[4 * e + 1]);
-      acc[4 * e + 2] = fmaf(a, v.z, acc[4 * e + 2]);
-      acc[4 * e + 3] = fmaf(a, v.w, acc[4 * e + 3]);
-    }
+    for (int e = 0; e < 4; ++e) v[e] = __ldg(reinterpret_cast<const float4*>(src0 + sp * sstride + 128 * e));
+    add(a, v);
   }
   __syncthreads();  // rope table
-  if (c0 >= kNope) {
+  // inverse RoPE on dims 448..511 (block e = 3, lanes 16..31: pairs (4 lane, +1), (4 lane + 2, +3))
+  if (lane >= (kNope - 384) / 4) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int pr = (c0 - kNope) / 2 + e;
+    for (int x = 0; x < 2; ++x) {
+      const int pr = (384 + 4 * lane - kNope) / 2 + x;
       const float cs = rope_c[pr], sn = rope_s[pr];
-      const float x = acc[2 * e], y = acc[2 * e + 1];
-      acc[2 * e] = x * cs - y * sn;
-      acc[2 * e + 1] = x * sn + y * cs;
+      const float u = acc[12 + 2 * x], y = acc[12 + 2 * x + 1];
+      acc[12 + 2 * x] = u * cs - y * sn;
+      acc[12 + 2 * x + 1] = u * sn + y * cs;
     }
   }
-  uint32_t o[8];
+  uint16_t* dst = out + ((int64_t)qi * n_heads + h) * kD + 4 * lane;
 #pragma unroll
-  for (int e = 0; e < 8; ++e)
-    o[e] = (uint32_t)f32_to_bf16_bits(acc[2 * e]) | ((uint32_t)f32_to_bf16_bits(acc[2 * e + 1]) << 16);
-  uint4* dst = reinterpret_cast<uint4*>(out + ((int64_t)qi * n_heads + h) * kD + c0);
-  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t lo = (uint32_t)f32_to_bf16_bits(acc[4 * e]) | ((uint32_t)f32_to_bf16_bits(acc[4 * e + 1]) << 16);
+    const uint32_t hi = (uint32_t)f32_to_bf16_bits(acc[4 * e + 2]) | ((uint32_t)f32_to_bf16_bits(acc[4 * e + 3]) << 16);
+    *reinterpret_cast<uint2*>(dst + 128 * e) = make_uint2(lo, hi);
+  }
 }
 
 }  // namespace
