@@ -322,7 +322,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         const uint32_t ph = (it / kStages) & 1;
         const int acc = it % kAcc;
         const uint32_t aph = (it / kAcc) & 1;
-        if (!sm100::mbar_wait(&S.tempty[acc], aph ^ 1, abort) || !sm100::mbar_wait(&S.full[s], ph, abort)) break;
+        if (!sm100::mbar_wait_poll(&S.tempty[acc], aph ^ 1, abort) || !sm100::mbar_wait_poll(&S.full[s], ph, abort))
+          break;
         sm100::tc_fence_after();
         Stage& st = S.st[s];
         const uint32_t sfb_col = tmem + kSfbCol + 4 * sl;
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         wq = q;
       }
       int ok = 1;
-      if (lane == 0) ok = sm100::mbar_wait(&S.tfull[acc], aph, abort);
+      if (lane == 0) ok = sm100::mbar_wait_poll(&S.tfull[acc], aph, abort);
       // no break on a failed wait: every warp of the warpgroup keeps walking
       // the same stages so that the histogram flushes' named barriers match;
       // after an abort every wait returns at once and no work is done
