@@ -152,15 +152,17 @@ def fp4_peak(bf16_peak, bf16_src):
     return bf16_peak * FP4_OVER_BF16, f"{bf16_src} bf16 x {FP4_OVER_BF16:g} (nominal fp4:bf16)"
 
 
-def dominant_roofline(w, kmean_ms, idx_bytes, step_bytes, hbm, bf16, traffic):
+def dominant_roofline(w, kmean_ms, amean_ms, idx_bytes, step_bytes, hbm, bf16, traffic):
     """Roofline entry of the step's dominant call.  hbm = (GB/s, source) and
     bf16 = (TFLOP/s, source) are the measured peaks.
 
-    CSA decode: the index call streams every visible key once, HBM-bound.
-    CSA prefill: the index call's MXFP4 contraction is tensor-bound (peak:
-    the measured BF16 peak times the nominal FP4:BF16 ratio).  HCA: the dense
-    attention, 4d flops per (head, row), is tensor-bound (BF16 peak; FP16
-    operands run at the BF16 rate)."""
+    The dominant call is the one that takes longer of the index call
+    (kmean_ms) and the attention (amean_ms; for HCA the dense attention is
+    the only timed call).  CSA decode: the index call streams every visible
+    key once, HBM-bound.  CSA prefill: the index call's MXFP4 contraction is
+    tensor-bound (peak: the FP4 peak measured live); the sparse attention,
+    4d flops per (head, attended row), is tensor-bound (BF16 peak; FP16
+    operands run at the BF16 rate).  HCA: the dense attention, likewise."""
     p = w["params"]
     sec = kmean_ms * 1e-3
     hbm_peak, hbm_src = hbm
@@ -178,11 +180,18 @@ def dominant_roofline(w, kmean_ms, idx_bytes, step_bytes, hbm, bf16, traffic):
                     "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": kmean_ms,
                     "fp4_tflops": fp4_ach, "fp4_peak": fp4_pk, "fp4_frac": fp4_ach / fp4_pk,
                     "fp4_peak_source": fp4_src}
-        return {"bound": "tensor", "kernel": "csa_index_topk", "achieved": fp4_ach, "peak": fp4_pk,
-                "unit": "TFLOP/s", "frac": fp4_ach / fp4_pk,
-                "peak_source": fp4_src, "traffic": traffic,
-                "algorithmic_flops_per_launch": fl, "launch_ms": kmean_ms,
-                "hbm_achieved_gbs": hbm_ach, "hbm_frac": hbm_ach / hbm_peak}
+        idx = {"bound": "tensor", "kernel": "csa_index_topk", "achieved": fp4_ach, "peak": fp4_pk,
+               "unit": "TFLOP/s", "frac": fp4_ach / fp4_pk,
+               "peak_source": fp4_src, "traffic": traffic,
+               "algorithmic_flops_per_launch": fl, "launch_ms": kmean_ms,
+               "hbm_achieved_gbs": hbm_ach, "hbm_frac": hbm_ach / hbm_peak}
+        if amean_ms <= kmean_ms:
+            return idx
+        fa = algorithmic_flops(w)
+        a_ach = fa / (amean_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "kernel": "csa_sparse_attn", "achieved": a_ach, "peak": bf16_peak,
+                "unit": "TFLOP/s", "frac": a_ach / bf16_peak, "peak_source": bf16_src, "traffic": None,
+                "algorithmic_flops_per_launch": fa, "launch_ms": amean_ms, "index_call": idx}
     fl = algorithmic_flops(w)
     ach = fl / sec / 1e12
     return {"bound": "tensor", "kernel": "hca_dense_attn", "achieved": ach, "peak": bf16_peak,
@@ -616,6 +625,8 @@ def run_config(config, args, world, rank, local):
                 ev[1].record(stream)
             stream.wait_stream(side0)
             dw.sparse_attn()
+            if ev is not None:
+                ev[2].record(stream)
         else:
             dw.compress()
             if ev is not None:
@@ -686,6 +697,8 @@ def run_config(config, args, world, rank, local):
             ev[1].record(stream)
         if g2 is not None:
             g2.replay()
+            if ev is not None:
+                ev[2].record(stream)
 
     for i in range(3):
         timed_step(i)
@@ -701,7 +714,7 @@ def run_config(config, args, world, rank, local):
         i += 1
     torch.cuda.synchronize()
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -714,7 +727,9 @@ def run_config(config, args, world, rank, local):
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1)
-    kern_ms = [a.elapsed_time(b) for a, b in evs]
+    kern_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    # CSA: the sparse attention (its graph replays right after the index call's)
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs] if p.k > 0 else kern_ms
     # a little more load for the clock sampler, then stop it (untimed)
     t_end = time.perf_counter() + 0.3
     while time.perf_counter() < t_end:
@@ -777,8 +792,9 @@ def run_config(config, args, world, rank, local):
     e2e_ms = e0.elapsed_time(e1) / n_e2e
 
     kmean = float(np.mean(kern_ms))
+    amean = float(np.mean(attn_ms))
     if world > 1:
-        ms, e2e_ms, kmean = max_over_ranks([ms, e2e_ms, kmean], "cuda")
+        ms, e2e_ms, kmean, amean = max_over_ranks([ms, e2e_ms, kmean, amean], "cuda")
     err = int(sum(d.err_bits() for d in dws))
 
     if rank != 0:
@@ -787,7 +803,7 @@ def run_config(config, args, world, rank, local):
     ms_per_step = ms / args.steps
     value = job_value(world, queries, ms_per_step)
     peak, peak_kind = measured_peaks()
-    roofline = dominant_roofline(w, kmean, idx_bytes, step_bytes, (peak, peak_kind), measured_tensor_peak(),
+    roofline = dominant_roofline(w, kmean, amean, idx_bytes, step_bytes, (peak, peak_kind), measured_tensor_peak(),
                                  recorded_traffic(f"csa_index_topk@{config}") if p.k > 0 else None)
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
@@ -802,6 +818,8 @@ def run_config(config, args, world, rank, local):
         "gpu_launches_source": "graph kernel nodes" if kernels_per_step is not None else "static count",
         "graphs": not args.no_graph,
         "roofline": roofline,
+        "calls_ms": ({"index_call_with_compress_beside": kmean, "attention": amean} if p.k > 0
+                     else {"dense_attention": kmean}),
         "step_roofline": step_roofline_entry(w, ms_per_step, step_bytes, peak, measured_tensor_peak()[0]),
         "e2e": {"value": job_value(world, queries, e2e_ms), "unit": "queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

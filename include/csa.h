@@ -220,6 +220,12 @@ csa_status csa_index_quantize(const csa_params* params, const void* x, int64_t n
  *   n_max     host upper bound on n_t over the batch (<= k_cap)
  *   out_idx   int32 [B][T][k]
  *   ws        workspace of csa_index_topk_workspace_bytes(params, T, n_max)
+ * Execution depends only on the shape and formats, never on the data:
+ * MXFP4 with 64 index heads of 128 dims and k_cap a multiple of 4 (each
+ * sequence's key-scale rows then start 16-byte aligned for TMA) runs on the
+ * tensor cores; every other accepted shape, k_cap not a multiple of 4
+ * included, runs on the CUDA cores.  Both compute the scores exactly when
+ * every partial sum is representable in fp32, and then agree bit for bit.
  * ---------------------------------------------------------------------- */
 csa_status csa_index_topk(const csa_params* params, const void* q_idx,
                           const uint8_t* q_idx_sf, const float* w,

@@ -108,19 +108,26 @@ def test_dominant_roofline_binds_the_right_roof():
     # CSA decode: the index call against HBM
     w = synth.config("c1", B=2, L=8192)
     _, idx_bytes = bench.algorithmic_bytes(w)
-    r = bench.dominant_roofline(w, 0.01, idx_bytes, 2 * idx_bytes, hbm, bf16, 123)
+    r = bench.dominant_roofline(w, 0.01, 0.005, idx_bytes, 2 * idx_bytes, hbm, bf16, 123)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 123
     assert r["achieved"] == pytest.approx(idx_bytes / 1e-5 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 6451.8)
     assert r["frac_vs_8tbs_datasheet"] == pytest.approx(r["achieved"] / 8000.0)
-    # CSA prefill: the indexer's MXFP4 contraction against 4x the BF16 peak
+    # CSA prefill, index call longer: the indexer's MXFP4 contraction
+    # against the FP4 peak (here, without a GPU to probe: 4x the BF16 peak)
     w = synth.config("c4", B=1, L=1024)
-    r = bench.dominant_roofline(w, 2.0, 1e6, 2e6, hbm, bf16, None)
-    assert r["bound"] == "tensor" and r["peak"] == pytest.approx(4 * 1655.5)
+    r = bench.dominant_roofline(w, 2.0, 1.0, 1e6, 2e6, hbm, bf16, None)
+    assert r["bound"] == "tensor" and r["peak"] == pytest.approx(4 * 1655.5) and r["kernel"] == "csa_index_topk"
     assert r["achieved"] == pytest.approx(bench.index_flops(w) / 2e-3 / 1e12)
+    # CSA prefill, attention longer: the sparse attention against the BF16
+    # peak, the index call's entry beside it
+    r = bench.dominant_roofline(w, 1.0, 3.0, 1e6, 2e6, hbm, bf16, None)
+    assert r["bound"] == "tensor" and r["kernel"] == "csa_sparse_attn" and r["peak"] == 1655.5
+    assert r["achieved"] == pytest.approx(bench.algorithmic_flops(w) / 3e-3 / 1e12)
+    assert r["index_call"]["kernel"] == "csa_index_topk"
     # HCA: the dense attention against the BF16 peak
     w = synth.config("c3", B=1, L=4096)
-    r = bench.dominant_roofline(w, 0.1, 0, 1e6, hbm, bf16, None)
+    r = bench.dominant_roofline(w, 0.1, 0.1, 0, 1e6, hbm, bf16, None)
     assert r["bound"] == "tensor" and r["peak"] == 1655.5 and r["kernel"] == "hca_dense_attn"
     assert r["achieved"] == pytest.approx(bench.algorithmic_flops(w) / 1e-4 / 1e12)
     s = bench.step_roofline_entry(w, 0.2, 1e6, 6451.8, 1655.5)
