@@ -76,6 +76,12 @@ struct ScoreKeys<true> {
   __device__ __forceinline__ static uint32_t sub(uint32_t key) { return key & 0xFu; }
 };
 
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 // exclusive scan of one int per thread over the 1024-thread block; returns
 // the prefix and writes the total to *total.  `tmp` holds >= 33 ints.
 __device__ __forceinline__ int block_scan_excl(int v, int* tmp, int* total) {
@@ -646,6 +652,114 @@ cudaError_t set_smem(K kernel, size_t bytes) {
   return set_max_smem(reinterpret_cast<const void*>(kernel), bytes);
 }
 
+// Histogram mode, rows of up to kFinishWords * 32 entries, steps 3-4 per
+// query, latency-trimmed: everything the step reads from global memory (the
+// row's selection bitmap, the tie list and its count, the second-level
+// histogram, the 4096-bin histogram) is requested at once, the tie
+// winners are marked in a shared-memory copy of the bitmap, and each warp
+// writes the indices of a contiguous run of bitmap words (lanes read
+// consecutive words; shuffle prefix sums place them).
+constexpr int kFinishWords = 8192;            // 262144 entries: 32 KB of bitmap in shared memory
+constexpr int kFinishPer = kFinishWords / kThreads;
+constexpr int kTiePer = kTieCap / kThreads;
+
+template <bool kB16>
+__global__ void __launch_bounds__(kThreads, 1) topk_chunk_finish_s(const void* __restrict__ scores, int ld,
+                                                                    int n_max, const uint32_t* __restrict__ ghist,
+                                                                    const int32_t* __restrict__ q_pos0, int T, int m,
+                                                                    int k, int32_t* __restrict__ out_idx,
+                                                                    const uint32_t* __restrict__ gbits,
+                                                                    const int* __restrict__ gtidx,
+                                                                    const uint32_t* __restrict__ gtkey,
+                                                                    const int* __restrict__ gcount,
+                                                                    const uint32_t* __restrict__ gh2) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BitSmem& S = *reinterpret_cast<BitSmem*>(smem_raw);
+  uint32_t* rbits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(BitSmem));  // the row's bitmap
+  pdl_wait();
+  pdl_trigger();
+  const int qi = blockIdx.x;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int n_t = visible_entries(q_pos0, T, m, qi, n_max);
+  const void* row = score_row<kB16>(scores, qi, ld);
+  int32_t* out = out_idx + (int64_t)qi * k;
+  if (n_t <= k) {
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n_t ? i : -1;
+    return;
+  }
+  const int words = (n_t + 31) / 32;
+  // all global reads issued up front, into registers
+  const uint32_t* gb = gbits + (int64_t)qi * (ld / 32);
+  uint32_t bw[kFinishPer];
+#pragma unroll
+  for (int j = 0; j < kFinishPer; ++j) {
+    const int w = threadIdx.x + kThreads * j;
+    bw[j] = w < words ? __ldcg(gb + w) : 0u;
+  }
+  const int gc = __ldcg(gcount + qi);
+  const int nl = min(gc, kTieCap);
+  int ti[kTiePer];
+  uint32_t tk[kTiePer];
+#pragma unroll
+  for (int j = 0; j < kTiePer; ++j) {
+    const int c = threadIdx.x + kThreads * j;
+    ti[j] = c < nl ? __ldcg(gtidx + (int64_t)qi * kTieCap + c) : 0;
+    tk[j] = c < nl ? __ldcg(gtkey + (int64_t)qi * kTieCap + c) : 0u;
+  }
+  const uint32_t h2v = threadIdx.x < kSub ? __ldcg(gh2 + (int64_t)qi * kSub + threadIdx.x) : 0u;
+  int bstar, cgt, ncand;
+  threshold_bin(ghist + (int64_t)qi * kScoreHistBins, k, S, &bstar, &cgt, &ncand);
+  const int nb = ncand - cgt;
+  if (bstar < 0 || nb > kTieCap || gc != nb) {
+    select_full<kB16>(row, n_t, k, out, S);
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < kFinishPer; ++j) {
+    const int w = threadIdx.x + kThreads * j;
+    if (w < words) rbits[w] = bw[j];
+  }
+#pragma unroll
+  for (int j = 0; j < kTiePer; ++j) {
+    const int c = threadIdx.x + kThreads * j;
+    if (c < nb) {
+      S.tidx[c] = ti[j];
+      S.tkey[c] = tk[j];
+    }
+  }
+  if (threadIdx.x < kSub) S.h2[threadIdx.x] = h2v;
+  __syncthreads();
+  resolve_ties<kB16>(nb, k - cgt, n_t, S, [&](int i) { atomicOr(rbits + (i >> 5), 1u << (i & 31)); });
+  __syncthreads();
+  // ordered output: warp wid owns words [w0, w1), walked in 32-word slabs
+  const int per_warp = ((words + kThreads / 32 - 1) / (kThreads / 32) + 31) & ~31;
+  const int w0 = min(words, wid * per_warp), w1 = min(words, w0 + per_warp);
+  int cnt = 0;
+  for (int w = w0 + lane; w < w1; w += 32) cnt += __popc(rbits[w]);
+  cnt = warp_sum_int(cnt);
+  int tot;
+  int pos = block_scan_excl(lane == 0 ? cnt : 0, S.tmp, &tot);
+  pos = __shfl_sync(0xffffffffu, pos, 0);
+  for (int wb = w0; wb < w1; wb += 32) {
+    const int w = wb + lane;
+    uint32_t word = w < w1 ? rbits[w] : 0u;
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int p = pos + incl - c;
+    while (word) {
+      const int e = __ffs(word) - 1;
+      word &= word - 1;
+      out[p++] = 32 * w + e;
+    }
+    pos += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
 // ---- no-histogram mode, rows of up to kCap entries: 256 threads per query ----
 //
 // Many queries with short rows (prefill): one 8-warp CTA per query, several
@@ -813,10 +927,17 @@ cudaError_t launch_topk_t(const csa_params& p, const void* scores, int ld, int n
   uint32_t* gtkey = reinterpret_cast<uint32_t*>(gtidx + (size_t)nq * kTieCap);
   const int chunks = (n_max + kChunk - 1) / kChunk;
   if ((e = set_smem(topk_chunk_pass<kB16>, smem)) != cudaSuccess) return e;
-  if ((e = set_smem(topk_chunk_finish<kB16>, smem)) != cudaSuccess) return e;
   e = launch_pdl(topk_chunk_pass<kB16>, dim3(nq, chunks), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0,
                  T, p.m, p.topk, gbits, gtidx, gtkey, gcount, gh2);
   if (e != cudaSuccess) return e;
+  if (ld / 32 <= kFinishWords) {
+    const size_t smem_s = smem + (size_t)kFinishWords * 4;
+    if ((e = set_smem(topk_chunk_finish_s<kB16>, smem_s)) != cudaSuccess) return e;
+    return launch_pdl(topk_chunk_finish_s<kB16>, dim3(nq), dim3(kThreads), smem_s, st, scores, ld, n_max, hist,
+                      q_pos0, T, p.m, p.topk, out_idx, (const uint32_t*)gbits, (const int*)gtidx,
+                      (const uint32_t*)gtkey, (const int*)gcount, (const uint32_t*)gh2);
+  }
+  if ((e = set_smem(topk_chunk_finish<kB16>, smem)) != cudaSuccess) return e;
   return launch_pdl(topk_chunk_finish<kB16>, dim3(nq), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T,
                     p.m, p.topk, out_idx, gbits, (const int*)gtidx, (const uint32_t*)gtkey, (const int*)gcount,
                     (const uint32_t*)gh2);

@@ -50,6 +50,7 @@ def _check(w, dw, queries=None):
     ("c1", dict(B=3, L=[16384, 9001, 4099])),                   # one CTA per query, ragged rows
     ("c1", dict(B=2, L=[200000, 131072 + 12])),                 # 50000 / 32771 entries: chunked rows
     ("c2", dict(B=2, L=262144, cluster=(1, 1024, 3.0))),        # 65536 entries, planted cluster, k = 1024
+    ("c1", dict(B=1, L=1200000)),                               # 300000 entries: bitmap beyond the finish's shared copy
 ])
 def test_topk_exact(fmt, name, kw):
     w = synth.with_score_fmt(synth.config(name, **kw), fmt)
@@ -68,10 +69,12 @@ def test_bf16_scores_are_the_rounded_exact_scores():
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-def test_topk_duplicate_keys_in_threshold_bin(fmt):
+@pytest.mark.parametrize("L", [32768, 200000])
+def test_topk_duplicate_keys_in_threshold_bin(fmt, L):
     """Every index key repeated 16 times: the threshold bin's ties come in
-    groups of equal scores that only the index order separates."""
-    w = synth.with_score_fmt(synth.config("c1", B=2, L=32768), fmt)
+    groups of equal scores that only the index order separates (one CTA per
+    row, and chunked rows)."""
+    w = synth.with_score_fmt(synth.config("c1", B=2, L=L), fmt)
     for key in ("k_idx", "k_idx_sf"):
         a = w[key]
         w[key] = np.ascontiguousarray(np.repeat(a[:, ::16], 16, axis=1)[:, :a.shape[1]])
