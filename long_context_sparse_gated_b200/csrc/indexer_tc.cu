@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
       sm100::prefetch_tmap(&tm_sfq);
       uint32_t it = 0, nq = 0;
       int bs = 0;
+      const uint64_t key_policy = sm100::l2_policy_evict_first();
       auto wk = make_walker<kPrefill>(n_queries, T, n_max);
       while (wk.next(q_pos0, T, m, n_max)) {
         if (wk.fresh) {  // the stage's query (pair): 64 heads each, once per query
@@ -288,8 +289,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) index_scores_tc(
         sm100::mbar_arrive_expect_tx(&S.full[s], M::kStageTx);
         const int64_t row = (int64_t)bs * k_cap + (int64_t)wk.j * M::kKeys;
 #pragma unroll
-        for (int g = 0; g < M::kT; ++g)
-          sm100::tma_load_3d(st.key[g], &tm_key, &S.full[s], 0, (int32_t)(row / 4) + g * (kTileM / 4), 0);
+        for (int g = 0; g < M::kT; ++g) {
+          const int32_t y = (int32_t)(row / 4) + g * (kTileM / 4);
+          // decode streams every key once: evict-first keeps the scores the
+          // selector reads next in L2; prefill re-reads a sequence's keys
+          if (kPrefill) sm100::tma_load_3d(st.key[g], &tm_key, &S.full[s], 0, y, 0);
+          else sm100::tma_load_3d_hint(st.key[g], &tm_key, &S.full[s], 0, y, 0, key_policy);
+        }
         sm100::tma_load_1d(st.sfk, &tm_sfk, &S.full[s], (int32_t)row);
         ++it;
       }

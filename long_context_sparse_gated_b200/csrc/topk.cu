@@ -38,6 +38,7 @@
 // writes the output; longer rows use the global-memory fallback.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -224,6 +225,9 @@ struct BitSmem {
   int tie_count, grp_count;
   int bstar, cgt, ncand;
 };
+
+// topk_fused stages its row's scores after BitSmem (32768 fp32 scores at most).
+constexpr size_t kRowStageOff = (sizeof(BitSmem) + 127) & ~size_t(127);
 
 // Global-memory fallback for a row (heavy ties): radix select over the
 // keys, then an ordered compaction, 1024 entries per step.
@@ -445,6 +449,10 @@ __global__ void __launch_bounds__(kThreads, 1) topk_fused(const void* __restrict
                                                            int32_t* __restrict__ out_idx) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BitSmem& S = *reinterpret_cast<BitSmem*>(smem_raw);
+  // the row's scores, copied into shared memory while the threshold bin is found
+  uint8_t* srow = smem_raw + kRowStageOff;
+  __shared__ uint64_t rbar;
+  __shared__ int rabort;
   pdl_wait();
   pdl_trigger();
   const int qi = blockIdx.x;
@@ -455,16 +463,35 @@ __global__ void __launch_bounds__(kThreads, 1) topk_fused(const void* __restrict
     for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n_t ? i : -1;
     return;
   }
+  const uint32_t row_bytes = ((uint32_t)n_t * (kB16 ? 2u : 4u) + 15u) & ~15u;  // within the row's ld padding
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&rbar, 1);
+    rabort = 0;
+    sm100::fence_mbar_init();
+  }
   if (threadIdx.x < kSub) S.h2[threadIdx.x] = 0u;
   if (threadIdx.x == 0) S.tie_count = 0;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    sm100::mbar_arrive_expect_tx(&rbar, row_bytes);
+    sm100::bulk_load(srow, row, row_bytes, &rbar);
+  }
   int bstar, cgt, ncand;
   threshold_bin(ghist + (int64_t)qi * kScoreHistBins, k, S, &bstar, &cgt, &ncand);
   const int nb = ncand - cgt;
+  // scores from shared memory once they have landed (from global memory if
+  // the copy timed out)
+  const bool staged = sm100::mbar_wait(&rbar, 0, &rabort);
+  if (!staged && threadIdx.x == 0) {
+    volatile int again = 0;  // the copy must not outlive the CTA: one more bounded wait
+    sm100::mbar_wait(&rbar, 0, &again);
+  }
+  const void* src = __syncthreads_and(staged) ? (const void*)srow : row;
   if (bstar < 0 || nb > kTieCap) {
     select_full<kB16>(row, n_t, k, out, S);
     return;
   }
-  scan_chunk<kB16>(row, 0, n_t, bstar, S.bits, kThreads, &S.tie_count, S.tidx, S.tkey, S.h2);
+  scan_chunk<kB16>(src, 0, n_t, bstar, S.bits, kThreads, &S.tie_count, S.tidx, S.tkey, S.h2);
   __syncthreads();
   if (S.tie_count != nb) {  // the histogram does not describe these scores
     select_full<kB16>(row, n_t, k, out, S);
@@ -914,8 +941,9 @@ cudaError_t launch_topk_t(const csa_params& p, const void* scores, int ld, int n
   }
   const size_t smem = sizeof(BitSmem);
   if (n_max <= kChunk) {
-    if ((e = set_smem(topk_fused<kB16>, smem)) != cudaSuccess) return e;
-    return launch_pdl(topk_fused<kB16>, dim3(nq), dim3(kThreads), smem, st, scores, ld, n_max, hist, q_pos0, T, p.m,
+    const size_t smem_f = kRowStageOff + (size_t)ld * (kB16 ? 2 : 4);
+    if ((e = set_smem(topk_fused<kB16>, smem_f)) != cudaSuccess) return e;
+    return launch_pdl(topk_fused<kB16>, dim3(nq), dim3(kThreads), smem_f, st, scores, ld, n_max, hist, q_pos0, T, p.m,
                       p.topk, out_idx);
   }
   // the counters and second-level histograms follow the per-query

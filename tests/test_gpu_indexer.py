@@ -101,3 +101,18 @@ def test_tc_prefill_query_pairs(score_fmt):
     got = dw.idx.cpu().numpy()
     for (b, tq), ref in idx.items():
         np.testing.assert_array_equal(got[b, tq], ref, err_msg=f"b={b} tq={tq}")
+
+
+@pytest.mark.parametrize("T,B", [(5, 3), (6, 1), (2, 4)])
+def test_tc_short_query_runs(T, B):
+    """The smallest prefill shapes (T = 5: two pairs and a single query per
+    sequence; T = 6: three pairs) and a multi-query decode (T = 2, one query
+    per stage): scores bit for bit and top-k sets equal the oracle's."""
+    w = synth.config("c1", B=B, L=[20000 + 97 * b for b in range(B)], T=T)
+    dw = _run_index(w)
+    g = _scores(dw)
+    idx, scores = pipeline.index_topk(w, return_scores=True)
+    got = dw.idx.cpu().numpy()
+    for (b, tq), sc in scores.items():
+        np.testing.assert_array_equal(g[b * T + tq, :len(sc)].astype(np.float64), sc, err_msg=f"b={b} tq={tq}")
+        np.testing.assert_array_equal(got[b, tq], idx[(b, tq)], err_msg=f"b={b} tq={tq}")
