@@ -8,16 +8,20 @@
 // One CTA = one query, one group of 64 heads, one split of its candidate
 // slots (entries, then window tokens), in 128-row tiles:
 //
-//   resolve   128 threads map the tile's slots to cache / window rows
-//   gather    the same threads each issue one 576-byte bulk copy (TMA
-//             engine, no tensor map) of their row into a staging area and
-//             load the row's scale; meanwhile the BF16 query (TMA) arrives
-//             and its amax is taken
-//   convert   the rows are read from the staging area, converted to FP16
-//             and stored as a 128-row x 512-dim K-major tile V' (128-byte
-//             swizzle); the query is converted in place to FP16 times 2^-e
-//             (e from its amax, so that it fits FP16 whatever its BF16
-//             range; 2^e joins the logit factor).
+//   resolve   128 threads map the tile's slots to cache / window row
+//             addresses (the next tile's selected entries are loaded at the
+//             start of a tile and resolved after its S MMAs are issued,
+//             when those rows are also prefetched into L2)
+//   gather    every thread loads its share of the tile (row 8 warp +
+//             lane/4, nine 16-byte chunks) and the row's scale straight into
+//             registers, before the wait for the previous tile's O MMAs;
+//             for the first tile the BF16 query (TMA) arrives meanwhile and
+//             each head's amax is taken
+//   convert   the four lanes of a row agree on its factors, convert it to
+//             FP16 and store it into a 128-row x 512-dim K-major tile V'
+//             (128-byte swizzle); the query is converted in place to FP16
+//             times 2^-e (e from its amax, so that it fits FP16 whatever its
+//             BF16 range; 2^e joins the logit factor).
 //   S^T       tcgen05.mma kind::f16 (FP16 A/B, FP32 accumulate):
 //             S^T[j, h] = sum_c V'[j, c] Q'[h, c]
 //             (M = 128 rows, N = 64 heads, K = 512) into TMEM, 32
@@ -35,8 +39,8 @@
 //             M = 128 dims x 4 blocks, N = 64 heads, K = 128 rows)
 //   epilogue  normalise (with the sink term when the split is the whole
 //             row set), inverse RoPE, then the 64 x 512 result is staged in
-//             shared memory and written with coalesced 16-byte stores: the
-//             BF16 output, or with several splits the fp32 partial O/l and
+//             shared memory and written with one bulk store: the BF16
+//             output, or with several splits the fp32 partial O/l and
 //             (m, l) that attn_merge_f32 combines in split order.
 //
 // Range.  Row j is stored as V'_j = v_j / c_j with c_j = s_j * 2^-k_j: the

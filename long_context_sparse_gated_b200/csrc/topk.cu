@@ -25,17 +25,20 @@
 //      exact threshold key and an index bitmap of the keys equal to it;
 //   4. one block scan over the bitmap's popcounts writes the selected
 //      indices in ascending order.
-// Rows of up to 32768 entries run as one CTA per query (topk_fused); longer
+// Rows of up to 32768 entries run as one CTA per query (topk_fused, which
+// copies the row's scores into shared memory while it runs step 1); longer
 // rows run steps 1-2 as one CTA per 32768-entry chunk (topk_chunk_pass,
 // bitmap and tie list in the workspace) and steps 1, 3, 4 as one CTA per
-// query (topk_chunk_finish).  When the threshold bin holds more than
-// kTieCap entries (heavy ties), the query falls back to a radix select read
-// from global memory and an ordered compaction.
+// query (topk_chunk_finish_s for rows up to 262144 entries, with the row's
+// bitmap in shared memory; topk_chunk_finish beyond).  When the threshold
+// bin holds more than kTieCap entries (heavy ties), the query falls back to
+// a radix select read from global memory and an ordered compaction.
 //
 // Without a histogram (the CUDA-core scorer, or more than 4096 queries in
-// a call), every entry of a row of up to kCap entries is staged in shared
-// memory, a radix select finds the k-th key and an ordered compaction
-// writes the output; longer rows use the global-memory fallback.
+// a call: prefill), rows of up to kCap entries run as one 256-thread CTA
+// each (topk_rows): the keys staged in shared memory, a radix select, an
+// ordered compaction by warp slabs.  Longer rows use a 1024-thread CTA
+// (topk_staged) and, beyond kCap, the global-memory fallback.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
